@@ -1,0 +1,356 @@
+#!/usr/bin/env python3
+"""Benchmark of the same-step KV chunk-attention hot path on B200.
+
+Workload (one "step"): one denoising step of one 880-token latent-frame chunk
+at the profile's steady state (1280x704 -> 40x22 tokens, 24 heads x 128, a
+2,640-token sink plus 18 ring slots = 18,480 keys), over 30 layers:
+per layer one pv_rope_append (3D RoPE of q, k and the append of k, v into the
+per-step ring) and one pv_chunk_attn, then one pv_euler_step on the chunk's
+48 x 44 x 80 latent.  Inputs are synthetic (seeded generator), the history of
+every layer is pre-filled, and the working set (6.9 GB of K/V) is far larger
+than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+W, HH, HEADS, D, R, LAYERS, STEP = 40, 22, 24, 128, 18, 30, 2
+T = W * HH
+CHUNK = 28                      # steady state: 17 earlier chunks + this one in the ring
+N_KEYS = (3 + R) * T            # 18,480
+LATENT = 48 * 44 * 80           # values of one latent frame
+ATTN_FLOPS = 4 * T * N_KEYS * HEADS * D          # one chunk_attn launch
+ROPE_BYTES = 6 * T * HEADS * D * 2               # q,k,v read; q_rot,k_rot,v written
+WORKLOAD = "steady chunk 880 q x 18480 k, 24x128, 30 layers + Euler 48x44x80"
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return json.load(fh), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("pv_attn.cu", "pv_internal.h", "pv_plan.cu"):
+        with open(os.path.join(ROOT, "same_step_kv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per chunk_attn launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "chunk_attn_880x18480.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    src = tb = None
+    for line in text.splitlines():
+        if line.startswith("source_hash:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            tb = float(line.split(":", 1)[1].strip())
+    return tb if (src == attn_source_hash() and tb) else None
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, p in zip(names, parts[3:7]):
+                if p.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def oracle_sample(seconds_hint=True):
+    """The fp64 oracle on one layer of the workload: RoPE of the chunk's q and k
+    and the attention of all 880 queries of all 24 heads over 18,480 keys.
+    Returns (flops, seconds, threads)."""
+    import numpy as np
+    import torch
+    from oracle import attention, rope
+    from same_step_kv_b200 import synth
+    q, k, v = synth.chunk_qkv(0, CHUNK, STEP, 0, T, HEADS, D)
+    kf, vf = synth.store_fill(0, 0, STEP, HEADS, N_KEYS, D)
+    q, k, v = (t.double().numpy() for t in (q, k, v))
+    K = kf.double().numpy().transpose(1, 0, 2).copy()
+    V = vf.double().numpy().transpose(1, 0, 2).copy()
+    t0 = time.perf_counter()
+    f, hh, ww = rope.token_coords(T, W, HH, 2 + CHUNK)
+    qr = rope.rotate(q, f, hh, ww)
+    kr = rope.rotate(k, f, hh, ww)
+    slot = (CHUNK - 1) % R
+    K[3 * T + slot * T: 3 * T + slot * T + T] = kr
+    V[3 * T + slot * T: 3 * T + slot * T + T] = v
+    attention.attend_heads(qr, K, V)
+    dt = time.perf_counter() - t0
+    return ATTN_FLOPS, dt, torch.get_num_threads()
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    vals = []
+    for i in range(args.warmup + args.steps):
+        fl, dt, thr = oracle_sample()
+        if i >= args.warmup:
+            vals.append(fl / dt / 1e12)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "chunk-attention TFLOP/s", "value": v,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": "one layer: RoPE + 880x18480 attention x 24 heads"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": "one of the 30 layers per step (880 queries x 24 heads x 18480 keys)"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "vs_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from same_step_kv_b200 import pv, synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+
+    # ---- setup: store with every layer's history at the steady state
+    cfg = pv.make_config(LAYERS, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
+    store = pv.KVStore(cfg, device=dev)
+    h = store.handle
+    st = pv.pv_kv_state()
+    st.phase, st.chunk = pv.PV_PHASE_STEADY, CHUNK
+    pv.pv_kv_set_state(h, 0, st)
+    Kr, Vr = store.k_region(), store.v_region()
+    for layer in range(LAYERS):
+        kf, vf = synth.store_fill(rank, layer, STEP, HEADS, N_KEYS, D, dev)
+        Kr[layer, STEP, 0] = kf
+        Vr[layer, STEP, 0] = vf
+    del kf, vf
+    qkv = [synth.chunk_qkv(rank, CHUNK, STEP, layer, T, HEADS, D, dev) for layer in range(LAYERS)]
+    q_rot = torch.empty(HEADS * T * D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, HEADS, D, dtype=torch.bfloat16, device=dev)
+    x = synth.latent(rank, 1, 48, 44, 80, dev).reshape(-1)
+    vel = synth.velocity(rank, CHUNK, STEP, LATENT, dev)
+    dsigma = 0.25 - 0.5
+
+    attn_ev = []
+
+    def step(record=False):
+        for layer in range(LAYERS):
+            q, k, v = qkv[layer]
+            pv.pv_rope_append(h, [0], layer, STEP, q, k, v, q_rot, cs)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+            pv.pv_chunk_attn(h, [0], layer, STEP, q_rot, out, None, cs)
+            if record:
+                e1.record(cs)
+                attn_ev.append((e0, e1))
+        pv.pv_euler_step(x, vel, LATENT, dsigma, cs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(cs)
+        for _ in range(args.steps):
+            step(record=True)
+        t1.record(cs)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        if rank == 0:
+            pass
+    ms_step = ms / args.steps
+
+    # ---- e2e: the same step through the public API from pinned host buffers
+    hq = [tuple(t.cpu().pin_memory() for t in qkv[l]) for l in range(LAYERS)]
+    hv = vel.cpu().pin_memory()
+    hx = x.cpu().pin_memory()
+    hres = torch.empty(LATENT, dtype=torch.float32).pin_memory()
+    dq = [tuple(torch.empty_like(t) for t in qkv[0]) for _ in range(2)]
+    dv = torch.empty_like(vel)
+    copy_s = torch.cuda.Stream(device=dev)
+    done = [torch.cuda.Event() for _ in range(2)]
+    used = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step():
+        with torch.cuda.stream(copy_s):
+            dv.copy_(hv, non_blocking=True)
+        for layer in range(LAYERS):
+            b = layer % 2
+            with torch.cuda.stream(copy_s):
+                if layer >= 2:
+                    copy_s.wait_event(used[b])
+                for dst, src in zip(dq[b], hq[layer]):
+                    dst.copy_(src, non_blocking=True)
+                done[b].record(copy_s)
+            cs.wait_event(done[b])
+            q, k, v = dq[b]
+            pv.pv_rope_append(h, [0], layer, STEP, q, k, v, q_rot, cs)
+            used[b].record(cs)
+            pv.pv_chunk_attn(h, [0], layer, STEP, q_rot, out, None, cs)
+        pv.pv_euler_step(x, dv, LATENT, dsigma, cs)
+        hres.copy_(x, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cs)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(cs)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = LAYERS * 3 * T * HEADS * D * 2 + LATENT * 4
+    d2h = LATENT * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        fl, dt, thr = oracle_sample()
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": "one of the 30 layers of a step: RoPE + 880x18480 attention, 24 heads"}
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        step_flops = LAYERS * ATTN_FLOPS * world
+        value = step_flops / (ms_step * 1e-3) / 1e12
+        achieved = ATTN_FLOPS / (attn_ms * 1e-3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        line = {
+            "metric": "chunk-attention TFLOP/s (whole step: 30 x rope_append + chunk_attn, Euler)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "heads": HEADS, "head_dim": D, "queries": T,
+                       "keys": N_KEYS, "layers": LAYERS,
+                       "l2": "inputs larger than L2 (6.9 GB of K/V per step), no flush"},
+            "latent_frames_per_s": world / (ms_step * 1e-3),
+            "pct_of_bf16_peak": 100.0 * value / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{src} bf16_tflops_sustained",
+                         "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
+                         "kernel": "attn_kernel<128> (pv_chunk_attn)",
+                         "ms_per_launch": attn_ms, "traffic": profiled_traffic()},
+            "e2e": {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (2 * LAYERS + 1),
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    store.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

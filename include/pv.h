@@ -1,0 +1,227 @@
+/*
+ * pv.h - same-step KV chunk attention for B200 (sm_100a), C ABI.
+ *
+ * The operation (PhysisServe Wan2.2-5B model card, "Inference profile" and
+ * the paragraph below it): video is generated chunk by chunk in latent space.
+ * The first chunk holds 3 latent frames, every later chunk 1 frame, and each
+ * chunk is denoised in 4 steps.  At denoising step s a chunk attends to the
+ * K/V that earlier chunks recorded at the same step s, plus a sink: the clean
+ * K/V of the first chunk, recorded by one extra pass at sigma = 0.  The
+ * history holds at most R recent chunks besides the sink.  Around the
+ * attention sit the 3D (frame, height, width) RoPE of q and k (blog
+ * "Learning Video Generation from the Wan2.2 Source Code", chapter 4, "3D
+ * RoPE") and the flow-matching Euler update x += (sigma_next - sigma) * v
+ * (same blog, chapter 5, "UniPC", and chapter 1).
+ *
+ * Conventions for every entry point
+ *  - Ownership: the caller allocates every device buffer and owns the CUDA
+ *    stream.  The library never allocates device memory; a pv_kv handle keeps
+ *    host bookkeeping and the caller's pointers only.
+ *  - Streams: `cuda_stream` is a cudaStream_t passed as void* (NULL = the
+ *    legacy default stream).  Every kernel call is asynchronous on it.
+ *  - Errors: every call returns a pv_status.  Arguments and shapes are
+ *    checked on the host before any launch; nothing aborts across the ABI.
+ *    A fault of an earlier asynchronous launch surfaces as PV_ERR_CUDA on a
+ *    later call.  pv_last_error() gives a one-line message for the calling
+ *    thread's most recent failure.
+ *  - Element types: "bf16" is IEEE bfloat16 (2 bytes), "f32" is float.
+ *  - Device pointers must be 16-byte aligned; the KV store must be 256-byte
+ *    aligned.
+ *  - Notation: T = frame_w * frame_h tokens per latent frame, F0 =
+ *    first_frames, R = ring_slots, H = heads, D = head_dim, Ltot = (F0 + R)*T
+ *    key rows per (layer, step, stream, head).
+ */
+#ifndef PV_H
+#define PV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PV_API __attribute__((visibility("default")))
+#else
+#define PV_API
+#endif
+
+typedef int pv_status;
+#define PV_OK                   0
+#define PV_ERR_INVALID_ARG      1  /* null pointer, bad enum, misaligned pointer */
+#define PV_ERR_SHAPE            2  /* sizes that the kernels do not support */
+#define PV_ERR_CAPACITY         3  /* a buffer smaller than required */
+#define PV_ERR_STATE            4  /* a call out of order in the chunk schedule */
+#define PV_ERR_UNSUPPORTED_ARCH 5  /* the current device is not sm_100 */
+#define PV_ERR_CUDA             6  /* a CUDA runtime or driver error */
+#define PV_ERR_TIMEOUT          7  /* a device-side wait gave up (see pv_kv_poll_device_error) */
+
+/* Step index of the sigma = 0 bootstrap pass that records the sink. */
+#define PV_STEP_SINK (-1)
+
+/* Largest ring (slots) and stream count that one handle supports. */
+#define PV_MAX_RING    64
+#define PV_MAX_STREAMS 64
+
+/* Phases of one stream (model card, "Inference profile"). */
+#define PV_PHASE_NEW    0  /* no chunk yet */
+#define PV_PHASE_FIRST  1  /* the first chunk (F0 frames) is being denoised */
+#define PV_PHASE_BOOT   2  /* the sigma = 0 pass over the clean first chunk */
+#define PV_PHASE_STEADY 3  /* chunks of one frame, reading sink + ring */
+
+/* Geometry and capacity of a KV store. */
+typedef struct pv_kv_config {
+    int layers;        /* transformer layers that keep a history (30 for Wan2.2-5B) */
+    int heads;         /* H */
+    int head_dim;      /* D: 64 or 128 */
+    int frame_w;       /* tokens per row of a latent frame (40 at 1280 px) */
+    int frame_h;       /* token rows of a latent frame (22 at 704 px) */
+    int first_frames;  /* F0: latent frames of the first chunk (3) */
+    int ring_slots;    /* R: recent chunks kept besides the sink (18), 1..PV_MAX_RING */
+    int steps;         /* denoising steps per chunk (4) */
+    int max_streams;   /* independent generation streams sharing the store */
+    int rope_pairs_t;  /* RoPE pairs of the time axis   (22 for D = 128, 12 for D = 64) */
+    int rope_pairs_h;  /* RoPE pairs of the height axis (21 for D = 128, 10 for D = 64) */
+    int rope_pairs_w;  /* RoPE pairs of the width axis  (21 for D = 128, 10 for D = 64) */
+    int max_frames;    /* largest latent-frame index + 1 that RoPE may see */
+    double rope_theta; /* RoPE base (10000) */
+} pv_kv_config;
+
+/* Host bookkeeping of one stream.  pv_kv_get_state fills it; pv_kv_set_state
+ * restores it (checkpoint / resume of the schedule position). */
+typedef struct pv_kv_state {
+    int phase;      /* PV_PHASE_* */
+    int chunk;      /* current chunk index j (0 = the first chunk, -1 before it) */
+    int fill;       /* ring slots holding a chunk: min(j, R) for j >= 1 */
+    int slot;       /* ring slot of the current chunk: (j - 1) mod R, or -1 */
+    int frame0;     /* latent-frame index of the current chunk's first frame */
+    int nframes;    /* latent frames in the current chunk */
+    int n_queries;  /* tokens of the current chunk: nframes * T */
+    int n_keys;     /* keys the current chunk reads at one step */
+    int slot_frame[PV_MAX_RING]; /* latent frame held by each slot, -1 if empty */
+} pv_kv_state;
+
+typedef struct pv_kv_s* pv_kv;
+
+/* Library version string (static storage). */
+PV_API const char* pv_version(void);
+
+/* Copies the calling thread's last error message into buf (always
+ * NUL-terminated when len > 0).  Returns the status of that failure. */
+PV_API pv_status pv_last_error(char* buf, size_t len);
+
+/* Sizes of the two caller-allocated device buffers for cfg.
+ *  kv_bytes: the KV store, 2 * layers * steps * max_streams * H * Ltot * D
+ *            bf16 (K region followed by V region).
+ *  ws_bytes: the workspace: RoPE cos/sin table, split-KV partial results,
+ *            arrival counters and a device error word. */
+PV_API pv_status pv_kv_required_bytes(const pv_kv_config* cfg, size_t* kv_bytes, size_t* ws_bytes);
+
+/* Creates a handle over caller buffers.  Checks cfg (D in {64,128}, RoPE
+ * pairs summing to D/2, 1 <= R <= PV_MAX_RING, ...), checks that the current
+ * device is sm_100, builds the RoPE table on the host in fp64, uploads it
+ * (synchronous cudaMemcpy) and zero-fills the store and the workspace
+ * (synchronous cudaMemset), so that unused key rows hold zeros.  All streams
+ * start in PV_PHASE_NEW.
+ * Passing kv_dev == NULL and ws_dev == NULL makes a bookkeeping-only handle:
+ * no device is touched, the schedule calls work, kernel calls return
+ * PV_ERR_STATE.  The handle is freed by pv_kv_destroy. */
+PV_API pv_status pv_kv_init(pv_kv* out, const pv_kv_config* cfg, void* kv_dev, size_t kv_bytes,
+                     void* ws_dev, size_t ws_bytes);
+PV_API pv_status pv_kv_destroy(pv_kv kv);
+
+/* Starts the next chunk of `stream` (model card, "Inference profile": the
+ * first chunk has F0 frames, every later one 1 frame).  NEW -> FIRST needs
+ * nframes == F0; BOOT or STEADY -> STEADY needs nframes == 1 and advances j,
+ * taking ring slot (j - 1) mod R.  Any other use returns PV_ERR_STATE and
+ * leaves the state unchanged. */
+PV_API pv_status pv_kv_begin_chunk(pv_kv kv, int stream, int nframes);
+
+/* Starts the sigma = 0 bootstrap pass of `stream` over its clean first chunk
+ * (model card: "receives an additional forward pass to build the persistent
+ * sink").  FIRST -> BOOT; any other phase returns PV_ERR_STATE. */
+PV_API pv_status pv_kv_begin_sink(pv_kv kv, int stream);
+
+PV_API pv_status pv_kv_get_state(pv_kv kv, int stream, pv_kv_state* out);
+/* Restores a state taken by pv_kv_get_state (fields are re-validated and the
+ * derived ones recomputed).  The store contents are the caller's to restore. */
+PV_API pv_status pv_kv_set_state(pv_kv kv, int stream, const pv_kv_state* st);
+
+/* Element offsets (in bf16 units from kv_dev) of key row `key` of
+ * (layer, step, stream, head) in the K and the V region.  step is 0..steps-1.
+ * Rows 0..F0*T-1 are the sink, row F0*T + slot*T + t is token t of a slot. */
+PV_API pv_status pv_kv_row_offset(pv_kv kv, int layer, int step, int stream, int head, int key,
+                           size_t* k_elem, size_t* v_elem);
+
+/* 3D RoPE of q and k plus the append of (k_rot, v) into the per-step store,
+ * for each listed stream at its current chunk.
+ *  streams[n_streams]: distinct stream ids (host array).
+ *  step: 0..steps-1, or PV_STEP_SINK for the bootstrap pass.
+ *    FIRST phase, step s: k_rot, v go to the sink rows of step buffer s.
+ *    PV_STEP_SINK (phase BOOT, see pv_kv_begin_sink): k_rot, v go to the
+ *      sink rows of every step buffer.
+ *    STEADY phase, step s: k_rot, v go to ring slot (j - 1) mod R of step s.
+ *  q, k, v: bf16 [sum_i Lq_i][H][D], the streams' tokens packed in list
+ *    order, Lq_i = nframes_i * T, tokens of a frame row-major (h * frame_w + w).
+ *  q_rot: bf16 output, head-major per stream: stream i's block starts at row
+ *    H * (sum_{i'<i} Lq_i') and is [H][Lq_i][D].
+ *  Token t of the chunk sits at latent frame frame0 + t / T, height
+ *  (t % T) / frame_w, width t % frame_w; pair p of a head rotates by
+ *  pos_axis(p) * theta^(-2 k / (2 * pairs_axis)), k = p's index in its axis
+ *  block, as the complex product (x[2p] + i x[2p+1]) e^{i angle}; fp32
+ *  arithmetic on a table built in fp64, rounded once to bf16. */
+PV_API pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer, int step,
+                         const void* q, const void* k, const void* v, void* q_rot,
+                         void* cuda_stream);
+
+/* Chunk attention of each listed stream at its current chunk, one launch:
+ *  o[q] = sum_k softmax_k(q_rot . k_rot / sqrt(D)) v_k over the stream's key
+ *  set at (layer, step): FIRST -> its own F0*T keys of step s; PV_STEP_SINK
+ *  (phase BOOT) -> its own clean keys; STEADY -> sink + the `fill` ring slots
+ *  of step s (F0*T + fill*T keys).  No causal mask.
+ *  q_rot: as written by pv_rope_append with the same stream list.
+ *  out: bf16 [sum_i Lq_i][H][D], token-major like q.
+ *  lse: optional f32 [sum_i Lq_i][H], natural-log log-sum-exp of the logits.
+ *  Computes in bf16 on the tensor cores with f32 accumulation and softmax. */
+PV_API pv_status pv_chunk_attn(pv_kv kv, int n_streams, const int* streams, int layer, int step,
+                        const void* q_rot, void* out, float* lse, void* cuda_stream);
+
+/* 3D RoPE over a whole clip of n_tokens = nframes * T tokens starting at
+ * latent frame frame0, with the handle's geometry and table (for full
+ * bidirectional attention over a video):
+ *  q, k, v: bf16 [n_tokens][H][D]; q_rot, k_rot, v_hm: bf16 [H][n_tokens][D]
+ *  (v_hm is v moved to head-major, unrotated). */
+PV_API pv_status pv_rope_dense(pv_kv kv, int n_tokens, int frame0, const void* q, const void* k,
+                        const void* v, void* q_rot, void* k_rot, void* v_hm, void* cuda_stream);
+
+/* Workspace bytes that pv_attn_dense needs for (Lq, Lk, H, D). */
+PV_API pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_dim, size_t* ws_bytes);
+
+/* Plain softmax attention on explicit head-major buffers, the same kernel as
+ * pv_chunk_attn:  q [H][n_q][D], k and v [H][n_k][D] bf16, out [n_q][H][D]
+ * bf16, lse optional f32 [n_q][H].  Key rows past n_k inside a 128-key tile
+ * are read from the next head (or as zeros past the buffer) and masked out,
+ * so k and v must hold finite values.
+ * ws: device workspace of pv_attn_dense_ws_bytes bytes, zero-filled by the
+ * caller before its first use (the kernels leave it zeroed again). */
+PV_API pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, int n_k,
+                        int heads, int head_dim, void* out, float* lse, void* ws,
+                        size_t ws_bytes, void* cuda_stream);
+
+/* Flow-matching Euler update in place (blog chapter 5, "UniPC"):
+ *  x[i] += dsigma * v[i] for i < n, f32, one fused multiply-add per element.
+ *  dsigma = sigma_next - sigma (negative while denoising), computed by the
+ *  caller in fp64 and passed rounded to f32. */
+PV_API pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* cuda_stream);
+
+/* Reads (synchronously) and clears the device error word that the kernels of
+ * this handle set when a bounded device-side wait gives up.  *code is 0 when
+ * no wait timed out. */
+PV_API pv_status pv_kv_poll_device_error(pv_kv kv, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PV_H */

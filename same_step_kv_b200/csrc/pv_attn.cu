@@ -1,0 +1,646 @@
+// Chunk attention on the 5th-generation tensor cores (sm_100a).
+//
+// o[q] = sum_k softmax_k(q . k / sqrt(D)) v_k over a contiguous range of key
+// rows, with the online softmax: the key range is walked in 128-key tiles,
+// keeping per query row a running maximum m and sum l, and rescaling the
+// output accumulator when m grows (PhysisServe Wan2.2-5B model card,
+// "Inference profile": the chunk's same-step key set; blog "Learning Video
+// Generation from the Wan2.2 Source Code", chapter 8: the two matrix
+// products QK^T and PV).
+//
+// One CTA = 3 warpgroups (12 warps):
+//   warp 0       TMA producer: the two Q tiles once, then K_j, V_j per key
+//                tile into a ring of shared-memory stages (128-byte swizzle).
+//   warp 1       allocates 512 TMEM columns; one lane issues every
+//                tcgen05.mma: S_X = Q_X K_j^T (SS form), O_X += P_X V_j (P
+//                from TMEM).
+//   warps 2, 3   idle.  Warpgroup 0 gives registers to the other two.
+//   warps 4..7   softmax of query tile A (TMEM lane = query row),
+//   warps 8..11  softmax of query tile B.
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [256+D,256+2D);
+// P_X (bf16 pairs) overwrites the first 64 columns of S_X.
+// The MMA order PV_A(j-1), S_A(j), PV_B(j-1), S_B(j) lets tile B's softmax run
+// while tile A's products are on the tensor pipe, and the other way round.
+// The running maximum is only moved when it grows by more than 8 (log2
+// units), so O is rescaled rarely; P stays below 2^8 and the final
+// normalisation uses the m that was actually applied, so the result is exact
+// softmax up to rounding.
+//
+// Every mbarrier wait is bounded (about one second); a wait that gives up
+// sets the device error word, makes the CTA skip its remaining work, waits
+// (bounded) for its own copies and MMAs, frees TMEM and returns.
+#include "pv_internal.h"
+
+namespace pv {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kRegsLow = 80;    // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsHigh = 208;  // softmax warpgroups after setmaxnreg.inc
+static_assert(kRegsLow * 128 + 2 * kRegsHigh * 128 <= 168 * kThreads, "register split");
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+
+template <int D>
+struct Cfg {
+    static constexpr int kSub = D / 64;                      // 64-column swizzle sub-tiles
+    static constexpr int kTileBytes = kQRows * D * 2;        // one 128-row tile
+    static constexpr int kStages = D == 128 ? 5 : 8;         // K/V ring depth
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    static constexpr int kSmem = kBarOff + 256 + 1024;       // + barriers + alignment slack
+    static constexpr uint32_t kColsO = 256;
+};
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_full[2];
+    uint64_t mma_done;
+    uint64_t kv_full[8];
+    uint64_t kv_empty[8];
+    uint32_t tmem_base;
+    int abort;
+    int last[2];
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// ----------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false when it gave up (the CTA is then aborting).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Bars* b, int* err) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try(bar, parity)) {
+        if (*(volatile int*)&b->abort) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            atomicExch(err, 1);
+            *(volatile int*)&b->abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// ----------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+#define PV_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
+                 "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define PV_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
+                 "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+
+// 32 / 128 consecutive TMEM columns of this thread's lane.  The wait for
+// the load sits in the same asm statement, so no use of the registers can be
+// scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        PV_W8(0), PV_W8(8), PV_W8(16), PV_W8(24)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        PV_W8(0), PV_W8(8)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: start, leading / stride byte offsets,
+// version 1 (sm_100), 128-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, f32 accumulator, A
+// K-major, B K-major or MN-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+struct Unit {
+    int si, head, qb, split, kt0, n_iter, q0, rows[2];
+};
+
+__device__ __forceinline__ Unit decode_unit(const AttnParams& p) {
+    Unit u{};
+    const int b = blockIdx.x;
+    for (int i = 0; i < p.n_streams; ++i) {
+        const AttnStreamDesc& s = p.st[i];
+        const int n = p.heads * s.n_qb * s.n_split;
+        if (b >= s.unit0 && b < s.unit0 + n) {
+            u.si = i;
+            int r = b - s.unit0;
+            u.split = r % s.n_split;
+            r /= s.n_split;
+            u.qb = r % s.n_qb;
+            u.head = r / s.n_qb;
+            u.kt0 = (int)((long long)u.split * s.n_kt / s.n_split);
+            u.n_iter = (int)((long long)(u.split + 1) * s.n_kt / s.n_split) - u.kt0;
+            u.q0 = u.qb * kQBlock;
+            u.rows[0] = min(kQRows, s.n_q - u.q0);
+            u.rows[1] = max(0, min(kQRows, s.n_q - u.q0 - kQRows));
+            return u;
+        }
+    }
+    u.si = -1;
+    return u;
+}
+
+// ----------------------------------------------------------------- roles
+template <int D>
+__device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                         const AttnParams& p, const Unit& u, uint8_t* smem, Bars* b) {
+    using C = Cfg<D>;
+    const AttnStreamDesc& s = p.st[u.si];
+    const int ntile = u.rows[1] > 0 ? 2 : 1;
+    const uint32_t qbar = smem_u32(&b->q_full);
+    mbar_expect_tx(qbar, ntile * C::kTileBytes);
+    const int qrow = s.q_row0 + u.head * s.n_q + u.q0;
+    for (int t = 0; t < ntile; ++t)
+        for (int c = 0; c < C::kSub; ++c)
+            tma_load(smem_u32(smem + C::kQOff + t * C::kTileBytes + c * 16384), tq, c * 64,
+                     qrow + t * kQRows, qbar);
+    const int krow0 = s.kv_row0 + u.head * s.kv_head_stride + u.kt0 * kKeyTile;
+    int issued = 0;
+    for (int j = 0; j < u.n_iter && !b->abort; ++j) {
+        for (int w = 0; w < 2; ++w) {
+            const int idx = 2 * j + w;
+            const int st = idx % C::kStages;
+            const uint32_t ph = (idx / C::kStages) & 1;
+            if (!mbar_wait(smem_u32(&b->kv_empty[st]), ph ^ 1, b, p.err)) break;
+            const uint32_t full = smem_u32(&b->kv_full[st]);
+            mbar_expect_tx(full, C::kTileBytes);
+            const CUtensorMap* m = w == 0 ? tk : tv;
+            for (int c = 0; c < C::kSub; ++c)
+                tma_load(smem_u32(smem + C::kKVOff + st * C::kTileBytes + c * 16384), m, c * 64,
+                         krow0 + j * kKeyTile, full);
+            issued = idx + 1;
+        }
+    }
+    // Before leaving, make sure no copy of ours is still landing in shared
+    // memory: wait (bounded) for the last load issued into each stage.
+    for (int idx = max(0, issued - C::kStages); idx < issued; ++idx) {
+        const int st = idx % C::kStages;
+        const uint32_t ph = (idx / C::kStages) & 1;
+        const uint32_t bar = smem_u32(&b->kv_full[st]);
+        const long long t0 = clock64();
+        while (!mbar_try(bar, ph) && clock64() - t0 < kWaitCycles) {
+        }
+    }
+    {
+        const long long t0 = clock64();
+        while (!mbar_try(qbar, 0) && clock64() - t0 < kWaitCycles) {
+        }
+    }
+}
+
+template <int D>
+__device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Bars* b,
+                           uint32_t tmem) {
+    using C = Cfg<D>;
+    constexpr uint32_t idesc_qk = idesc_bf16(kQRows, kKeyTile, false);
+    constexpr uint32_t idesc_pv = idesc_bf16(kQRows, D, true);
+    const bool hasB = u.rows[1] > 0;
+    const uint32_t sQ = smem_u32(smem + C::kQOff);
+    const uint32_t sKV = smem_u32(smem + C::kKVOff);
+    auto qk = [&](int X, int stage) {
+        const uint32_t tS = tmem + X * 128;
+        const uint32_t qa = sQ + X * C::kTileBytes;
+        const uint32_t kb = sKV + stage * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tS, sdesc(qa + off, 16, 1024), sdesc(kb + off, 16, 1024), idesc_qk, kk > 0);
+        }
+    };
+    auto pv = [&](int X, int stage, bool acc) {
+        const uint32_t tS = tmem + X * 128;
+        const uint32_t tO = tmem + C::kColsO + X * D;
+        const uint32_t vb = sKV + stage * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kKeyTile / 16; ++kk)
+            mma_ts(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
+                   (acc || kk > 0) ? 1u : 0u);
+    };
+    bool ok = mbar_wait(smem_u32(&b->q_full), 0, b, p.err);
+    tc_fence_after();
+    const int n = u.n_iter;
+    for (int j = 0; ok && j < n; ++j) {
+        const int ks = (2 * j) % C::kStages;
+        const uint32_t kph = ((2 * j) / C::kStages) & 1;
+        const int vs_prev = (2 * j - 1 + C::kStages) % C::kStages;
+        const uint32_t vph_prev = ((2 * j - 1) / C::kStages) & 1;
+        if (j > 0) {
+            ok = mbar_wait(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
+                 mbar_wait(smem_u32(&b->p_full[0]), (j - 1) & 1, b, p.err);
+            if (!ok) break;
+            tc_fence_after();
+            pv(0, vs_prev, j > 1);
+        }
+        if (!(ok = mbar_wait(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
+        tc_fence_after();
+        qk(0, ks);
+        tc_commit(smem_u32(&b->s_full[0]));
+        if (hasB) {
+            if (j > 0) {
+                if (!(ok = mbar_wait(smem_u32(&b->p_full[1]), (j - 1) & 1, b, p.err))) break;
+                tc_fence_after();
+                pv(1, vs_prev, j > 1);
+            }
+            qk(1, ks);
+            tc_commit(smem_u32(&b->s_full[1]));
+        }
+        if (j > 0) tc_commit(smem_u32(&b->kv_empty[vs_prev]));
+        tc_commit(smem_u32(&b->kv_empty[ks]));
+    }
+    if (ok) {
+        const int vs = (2 * n - 1) % C::kStages;
+        const uint32_t vph = ((2 * n - 1) / C::kStages) & 1;
+        ok = mbar_wait(smem_u32(&b->kv_full[vs]), vph, b, p.err) &&
+             mbar_wait(smem_u32(&b->p_full[0]), (n - 1) & 1, b, p.err);
+        if (ok) {
+            tc_fence_after();
+            pv(0, vs, n > 1);
+            tc_commit(smem_u32(&b->o_full[0]));
+            if (hasB && (ok = mbar_wait(smem_u32(&b->p_full[1]), (n - 1) & 1, b, p.err))) {
+                tc_fence_after();
+                pv(1, vs, n > 1);
+                tc_commit(smem_u32(&b->o_full[1]));
+            }
+            tc_commit(smem_u32(&b->kv_empty[vs]));
+        }
+    }
+    // every MMA issued by this thread has completed once mma_done flips
+    tc_commit(smem_u32(&b->mma_done));
+    const long long t0 = clock64();
+    while (!mbar_try(smem_u32(&b->mma_done), 0) && clock64() - t0 < kWaitCycles) {
+    }
+}
+
+template <int D>
+__device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, uint32_t tmem,
+                                 int X) {
+    using C = Cfg<D>;
+    const AttnStreamDesc& s = p.st[u.si];
+    const int wq = (threadIdx.x / 32) & 3;          // TMEM lane quadrant of this warp
+    const int r = wq * 32 + (threadIdx.x & 31);     // query row inside the tile
+    const uint32_t lane = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane + X * 128;
+    const uint32_t tO = tmem + lane + C::kColsO + X * D;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY;  // maximum applied to the exponentials, log2 units
+    float l = 0.f;        // sum of the exponentials
+    bool ok = true;
+    for (int j = 0; j < u.n_iter; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->s_full[X]), j & 1, b, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld128_wait(tS, sr);
+        const int valid = s.n_k - (u.kt0 + j) * kKeyTile;
+        if (valid < kKeyTile) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = __uint_as_float(sr[0]);
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+        const float m_new = fmaxf(m, mx * sl2);
+        const bool need = m_new > m + 8.0f;
+        // tcgen05.ld / st are warp-collective: rescale when any lane needs it
+        if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2(m - m_new) : 1.0f;  // 0 on the first tile
+            if (need) {
+                l *= alpha;
+                m = m_new;
+            }
+            if (j > 0) {
+                // O holds P V of tiles < j, complete: S(j) was committed after it
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tO + c, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + c, o);
+                }
+            }
+        }
+        float sum = 0.f;
+        const float nm = -m;
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float p0 = ex2(fmaf(__uint_as_float(sr[c + i]), sl2, nm));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[c + i + 1]), sl2, nm));
+                sum += p0 + p1;
+                pk[i / 2] = pack_bf16(p0, p1);
+            }
+            tmem_st16(tS + c / 2, pk);
+        }
+        l += sum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&b->p_full[X]));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->o_full[X]), 0, b, p.err));
+    if (ok) tc_fence_after();
+
+    // ---------------------------------------------------------- epilogue
+    const bool row_ok = ok && r < u.rows[X];
+    const int tok = s.out_tok0 + u.q0 + X * kQRows + r;
+    const float ln2 = 0.69314718055994531f;
+    if (s.n_split == 1) {
+        const float inv = 1.0f / l;
+        bf16* dst = p.out + ((size_t)tok * p.heads + u.head) * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            if (ok) {
+                tmem_ld32_wait(tO + c, o);
+            }
+            if (row_ok) {
+                uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int q = i * 8;
+                    d4[i] = make_uint4(
+                        pack_bf16(__uint_as_float(o[q + 0]) * inv, __uint_as_float(o[q + 1]) * inv),
+                        pack_bf16(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv),
+                        pack_bf16(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv),
+                        pack_bf16(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv));
+                }
+            }
+        }
+        if (row_ok && p.lse) p.lse[(size_t)tok * p.heads + u.head] = (m + __log2f(l)) * ln2;
+        return;
+    }
+
+    // split-KV: store the unnormalised partial, the last of the parts merges
+    const size_t slot_f = partial_slot_floats(D);
+    const int tile_id = (u.head * s.n_qb + u.qb) * kQTilesPerCta + X;
+    const size_t slot0 = (size_t)s.part0 + (size_t)tile_id * s.n_split;
+    float* mine = p.partial + (slot0 + u.split) * slot_f;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        if (ok) {
+            tmem_ld32_wait(tO + c, o);
+        }
+        if (row_ok) {
+            float4* d4 = reinterpret_cast<float4*>(mine + (size_t)r * D + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                    __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+        }
+    }
+    if (row_ok) {
+        mine[(size_t)kQRows * D + r] = m;
+        mine[(size_t)kQRows * D + kQRows + r] = l;
+    }
+    __threadfence();
+    named_sync(1 + X, 128);
+    if (r == 0) {
+        int last = 0;
+        if (ok && !*(volatile int*)&b->abort) {
+            int* cnt = p.counters + s.cnt0 + tile_id;
+            const int old = atomicAdd(cnt, 1);
+            last = old == s.n_split - 1;
+            if (last) *cnt = 0;  // ready for the next launch
+        }
+        b->last[X] = last;
+    }
+    named_sync(1 + X, 128);
+    if (!b->last[X] || !row_ok) return;
+    __threadfence();
+    float M = -INFINITY;
+    for (int i = 0; i < s.n_split; ++i)
+        M = fmaxf(M, __ldcg(p.partial + (slot0 + i) * slot_f + (size_t)kQRows * D + r));
+    float L = 0.f;
+    for (int i = 0; i < s.n_split; ++i) {
+        const float* pi = p.partial + (slot0 + i) * slot_f;
+        L += __ldcg(pi + (size_t)kQRows * D + kQRows + r) * ex2(__ldcg(pi + (size_t)kQRows * D + r) - M);
+    }
+    const float invL = 1.0f / L;
+    bf16* dst = p.out + ((size_t)tok * p.heads + u.head) * D;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 8) {
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int i = 0; i < s.n_split; ++i) {
+            const float* pi = p.partial + (slot0 + i) * slot_f;
+            const float w = ex2(__ldcg(pi + (size_t)kQRows * D + r) - M) * invL;
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(pi + (size_t)r * D + c));
+            const float4 bq = __ldcg(reinterpret_cast<const float4*>(pi + (size_t)r * D + c + 4));
+            acc[0] = fmaf(w, a.x, acc[0]);
+            acc[1] = fmaf(w, a.y, acc[1]);
+            acc[2] = fmaf(w, a.z, acc[2]);
+            acc[3] = fmaf(w, a.w, acc[3]);
+            acc[4] = fmaf(w, bq.x, acc[4]);
+            acc[5] = fmaf(w, bq.y, acc[5]);
+            acc[6] = fmaf(w, bq.z, acc[6]);
+            acc[7] = fmaf(w, bq.w, acc[7]);
+        }
+        *reinterpret_cast<uint4*>(dst + c) =
+            make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                       pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+    }
+    if (p.lse) p.lse[(size_t)tok * p.heads + u.head] = (M + __log2f(L)) * ln2;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams p) {
+    using C = Cfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Bars* b = reinterpret_cast<Bars*>(smem + C::kBarOff);
+    const Unit u = decode_unit(p);
+    if (u.si < 0) return;  // the same for every thread of the CTA
+    const int warp = threadIdx.x / 32;
+    const int lane_id = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&b->q_full), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&b->s_full[x]), 1);
+            mbar_init(smem_u32(&b->p_full[x]), 128);
+            mbar_init(smem_u32(&b->o_full[x]), 1);
+        }
+        mbar_init(smem_u32(&b->mma_done), 1);
+        for (int i = 0; i < C::kStages; ++i) {
+            mbar_init(smem_u32(&b->kv_full[i]), 1);
+            mbar_init(smem_u32(&b->kv_empty[i]), 1);
+        }
+        b->abort = 0;
+        b->last[0] = b->last[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&b->tmem_base)),
+                     "r"(512u)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = b->tmem_base;
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+        if (warp == 0) {
+            if (lane_id == 0) producer<D>(&tq, &tk, &tv, p, u, smem, b);
+        } else if (warp == 1) {
+            if (lane_id == 0) mma_issuer<D>(p, u, smem, b, tmem);
+            __syncwarp();
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+        const int X = warp / 4 - 1;
+        if (X == 0 || u.rows[1] > 0) softmax_epilogue<D>(p, u, b, tmem, X);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u)
+                     : "memory");
+    }
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const AttnParams& p, int n_units, cudaStream_t s) {
+    using C = Cfg<D>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    attn_kernel<D><<<n_units, kThreads, C::kSmem, s>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnParams& p, int n_units, cudaStream_t s) {
+    if (n_units <= 0) return cudaErrorInvalidValue;
+    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, p, n_units, s);
+    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, p, n_units, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pv

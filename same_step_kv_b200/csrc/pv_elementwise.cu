@@ -1,0 +1,139 @@
+// HBM-bound kernels: 3D RoPE + same-step KV append, and the Euler update.
+#include "pv_internal.h"
+
+namespace pv {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream(const bf16* p) {
+    // read once: do not keep in L1
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void st16(bf16* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+__device__ __forceinline__ float2 unpack(uint32_t w) {
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&w);
+    return __bfloat1622float2(b);
+}
+
+__device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Blog "Learning Video Generation from the Wan2.2 Source Code", chapter 4,
+// "3D RoPE": pair p of a head belongs to the time, height or width block and
+// turns by that coordinate times the pair's frequency, as the complex product
+// (x + i y) e^{i angle}.  One thread handles 8 consecutive dimensions (4
+// pairs, one 16-byte vector) of one (token, head) of q, k and v; rows are
+// read and written with 128-bit coalesced accesses.
+__global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant__ RopeParams p) {
+    const RopeStreamDesc& sd = p.st[blockIdx.y];
+    const int G = p.head_dim >> 3;                   // 16-byte groups per head row
+    const int per_tok = p.heads * G;
+    const int n_items = sd.n_tok * per_tok;
+    const int T = p.frame_w * p.frame_h;
+    for (int it = blockIdx.x * blockDim.x + threadIdx.x; it < n_items; it += gridDim.x * blockDim.x) {
+        const int t = it / per_tok;
+        const int j = it - t * per_tok;
+        const int h = j / G;
+        const int g = j - h * G;
+        const size_t in_off = ((size_t)(sd.in_tok0 + t) * p.heads + h) * p.head_dim + g * 8;
+        const uint4 qv = ld_stream(p.q + in_off);
+        const uint4 kv = ld_stream(p.k + in_off);
+        const uint4 vv = ld_stream(p.v + in_off);
+        const int f = sd.frame0 + t / T;
+        const int r = t % T;
+        const int hh = r / p.frame_w;
+        const int ww = r - hh * p.frame_w;
+        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t qo[4], ko[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int pair = g * 4 + u;
+            int idx;
+            if (pair < p.pairs_t) {
+                idx = f * p.pairs_t + pair;
+            } else if (pair < p.pairs_t + p.pairs_h) {
+                idx = p.tab_h0 + hh * p.pairs_h + (pair - p.pairs_t);
+            } else {
+                idx = p.tab_w0 + ww * p.pairs_w + (pair - p.pairs_t - p.pairs_h);
+            }
+            const float2 cs = __ldg(p.table + idx);
+            const float2 a = unpack(qw[u]);
+            const float2 b = unpack(kw[u]);
+            qo[u] = pack(fmaf(a.x, cs.x, -a.y * cs.y), fmaf(a.x, cs.y, a.y * cs.x));
+            ko[u] = pack(fmaf(b.x, cs.x, -b.y * cs.y), fmaf(b.x, cs.y, b.y * cs.x));
+        }
+        const size_t qrow = (size_t)sd.qrot_row0 + (size_t)h * sd.n_tok + t;
+        st16(p.q_rot + qrow * p.head_dim + g * 8, make_uint4(qo[0], qo[1], qo[2], qo[3]));
+        const uint4 kout = make_uint4(ko[0], ko[1], ko[2], ko[3]);
+        for (int d = 0; d < sd.n_dst; ++d) {
+            const size_t row = (size_t)sd.dst_row0[d] + (size_t)h * p.dst_head_stride + t;
+            st16(p.k_dst + row * p.head_dim + g * 8, kout);
+            st16(p.v_dst + row * p.head_dim + g * 8, vv);
+        }
+    }
+}
+
+// Blog chapter 5 ("UniPC"): the first-order Euler step x <- x + dsigma * v
+// with dsigma = sigma_next - sigma.  float4 path over the aligned body, a
+// scalar path for the ragged head and tail.
+__global__ void __launch_bounds__(256) euler_kernel(float* __restrict__ x,
+                                                    const float* __restrict__ v, size_t n,
+                                                    float dsigma) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool vec = ((((uintptr_t)x) | ((uintptr_t)v)) & 15) == 0;
+    if (vec) {
+        const size_t n4 = n >> 2;
+        float4* x4 = reinterpret_cast<float4*>(x);
+        const float4* v4 = reinterpret_cast<const float4*>(v);
+        for (size_t i = tid; i < n4; i += stride) {
+            float4 a = x4[i];
+            const float4 b = __ldcs(v4 + i);
+            a.x = fmaf(dsigma, b.x, a.x);
+            a.y = fmaf(dsigma, b.y, a.y);
+            a.z = fmaf(dsigma, b.z, a.z);
+            a.w = fmaf(dsigma, b.w, a.w);
+            x4[i] = a;
+        }
+        for (size_t i = (n4 << 2) + tid; i < n; i += stride) x[i] = fmaf(dsigma, v[i], x[i]);
+    } else {
+        for (size_t i = tid; i < n; i += stride) x[i] = fmaf(dsigma, v[i], x[i]);
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+}  // namespace
+
+cudaError_t launch_rope(const RopeParams& p, int max_tok, cudaStream_t s) {
+    const long long items = (long long)max_tok * p.heads * (p.head_dim / 8);
+    if (items >= (1LL << 31)) return cudaErrorInvalidValue;
+    // grid: enough CTAs per stream to cover the SMs a few times over
+    const int per_stream = (int)std::min<long long>((items + 255) / 256,
+                                                    std::max(1, 8 * sm_count() / p.n_streams));
+    dim3 grid(per_stream, p.n_streams);
+    rope_append_kernel<<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaStream_t s) {
+    const size_t want = (n / 4 + 255) / 256;
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>(want, (size_t)sm_count() * 8));
+    euler_kernel<<<grid, 256, 0, s>>>(x, v, n, dsigma);
+    return cudaGetLastError();
+}
+
+}  // namespace pv

@@ -1,0 +1,100 @@
+// Internal declarations shared by the host API and the kernels of libpv.
+// Nothing here is part of the C ABI (include/pv.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pv.h"
+
+namespace pv {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kMaxSteps = 8;              // denoising steps per chunk a handle may hold
+constexpr int kQRows = 128;               // query rows per tensor-core tile (MMA M)
+constexpr int kQTilesPerCta = 2;          // two query tiles share each K/V tile
+constexpr int kQBlock = kQRows * kQTilesPerCta;
+constexpr int kKeyTile = 128;             // keys per K/V tile (MMA N of Q K^T)
+constexpr int kMaxSplit = 32;             // split-KV parts of one query tile
+
+// ---------------------------------------------------------------- RoPE + append
+struct RopeStreamDesc {
+    int in_tok0;                     // first token of this stream in the packed input
+    int n_tok;                       // tokens of the chunk
+    int frame0;                      // latent frame of token 0
+    int n_dst;                       // K/V destinations (0: none, 1: a step, steps: sink pass)
+    long long qrot_row0;             // q_rot row (of D elements) of head 0, token 0
+    long long dst_row0[kMaxSteps];   // K/V-region row of head 0, token 0, per destination
+};
+
+struct RopeParams {
+    const bf16* q;
+    const bf16* k;
+    const bf16* v;
+    bf16* q_rot;
+    bf16* k_dst;            // K region base (store) or k_rot (dense)
+    bf16* v_dst;            // V region base (store) or v head-major (dense)
+    const float2* table;    // cos, sin per (axis, position, pair)
+    int heads, head_dim, frame_w, frame_h;
+    int pairs_t, pairs_h, pairs_w;
+    int tab_h0, tab_w0;     // table offsets of the height and width blocks
+    long long dst_head_stride;  // destination rows between heads
+    int n_streams;
+    RopeStreamDesc st[PV_MAX_STREAMS];
+};
+
+cudaError_t launch_rope(const RopeParams& p, int max_tok, cudaStream_t s);
+
+// ----------------------------------------------------------------- attention
+struct AttnStreamDesc {
+    int n_q;             // queries of this stream (per head)
+    int n_k;             // keys (per head)
+    int q_row0;          // q_rot row of head 0, query 0 (per head + n_q)
+    int kv_row0;         // K/V row of head 0, key 0
+    int kv_head_stride;  // K/V rows between heads
+    int out_tok0;        // first token row of out / lse
+    int n_qb;            // query blocks of kQBlock rows
+    int n_kt;            // key tiles
+    int n_split;         // key-range parts per query block
+    int unit0;           // first CTA index of this stream
+    int part0;           // first partial-result slot
+    int cnt0;            // first arrival counter
+};
+
+struct AttnParams {
+    bf16* out;
+    float* lse;
+    float* partial;      // split-KV partial results (unnormalised O, m, l)
+    int* counters;       // arrivals per query tile; the last arriver resets to 0
+    int* err;            // device error word (bounded waits that gave up)
+    int heads;
+    int head_dim;
+    float scale_log2;    // log2(e) / sqrt(D)
+    int n_streams;
+    AttnStreamDesc st[PV_MAX_STREAMS];
+};
+
+// Bytes of one partial-result slot for head dimension D.
+__host__ __device__ inline size_t partial_slot_floats(int D) { return (size_t)kQRows * D + 2 * kQRows; }
+
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnParams& p, int n_units, cudaStream_t s);
+
+// ----------------------------------------------------------------- Euler
+cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaStream_t s);
+
+// ----------------------------------------------------------------- host helpers
+// Encodes a 2D bf16 tensor map over `rows` rows of `D` elements with a
+// 64-element x 128-row box and the 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, char* err,
+                     size_t errlen);
+
+// Split-KV plan for one attention launch: fills n_split, unit0, part0, cnt0.
+// Returns the number of CTAs, or -1 when the partial slots do not suffice.
+int plan_attention(AttnStreamDesc* st, int n_streams, int heads, int n_sm, int part_capacity,
+                   int cnt_capacity, int* order);
+
+}  // namespace pv

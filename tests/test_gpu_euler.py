@@ -1,0 +1,60 @@
+"""Euler update on the GPU against the fp64 oracle (blog chapter 5, UniPC)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import f64
+from oracle import euler
+from same_step_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+FRAME = 48 * 44 * 80  # 168,960 latent values per frame
+
+
+@pytest.fixture(scope="module")
+def pv():
+    from same_step_kv_b200 import pv as m
+    return m
+
+
+@pytest.mark.parametrize("n,offset", [(1, 0), (7, 0), (1000, 1), (FRAME, 0), (FRAME + 3, 1),
+                                      (248 * FRAME, 0)])
+def test_euler_step_matches_oracle(pv, n, offset):
+    x = synth.normal_f32(101, (n + offset,), "cuda")
+    v = synth.normal_f32(102, (n + offset,), "cuda")
+    x_host = f64(x)[offset:]
+    v_host = f64(v)[offset:]
+    for sigma, nxt in zip(euler.SIGMAS_4[:-1], euler.SIGMAS_4[1:]):
+        ref = euler.euler_step(x_host, v_host, sigma, nxt)
+        pv.pv_euler_step(x[offset:], v[offset:], n, float(nxt - sigma))
+        torch.cuda.synchronize()
+        got = f64(x)[offset:]
+        err = np.abs(got - ref)
+        assert np.linalg.norm(got - ref) <= 1e-5 * np.linalg.norm(ref)
+        assert np.all(err <= 1e-5 * (np.abs(x_host) + np.abs((nxt - sigma) * v_host)) + 1e-30)
+        x_host = ref
+    if offset:
+        assert float(x[0]) == float(synth.normal_f32(101, (1,))[0])  # untouched prefix
+
+
+def test_euler_straight_line_closed_form(pv):
+    # v = x1 - x0 constant: four steps from sigma = 1 reach x0 (blog chapter 1)
+    n = 3 * FRAME
+    x0 = synth.normal_f32(103, (n,), "cuda")
+    x1 = synth.normal_f32(104, (n,), "cuda")
+    v = x1 - x0
+    x = x1.clone()
+    s = euler.SIGMAS_4
+    for i in range(4):
+        pv.pv_euler_step(x, v, n, float(s[i + 1] - s[i]))
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(x - x0)).item() <= 4e-6 * torch.max(torch.abs(x1) + torch.abs(x0)).item()
+
+
+def test_euler_rejects_bad_arguments(pv):
+    x = torch.zeros(8, device="cuda")
+    with pytest.raises(pv.PVError):
+        pv.pv_euler_step(x, 0, 8, -0.25)
+    with pytest.raises(pv.PVError):
+        pv.pv_euler_step(x, x, 8, float("nan"))
+    pv.pv_euler_step(x, x, 0, -0.25)  # empty is a no-op
