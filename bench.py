@@ -89,7 +89,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -129,9 +129,9 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-def oracle_sample(seconds_hint=True):
+def oracle_sample(heads=HEADS):
     """The fp64 oracle on one layer of the workload: RoPE of the chunk's q and k
-    and the attention of all 880 queries of all 24 heads over 18,480 keys.
+    and the attention of all 880 queries of `heads` heads over 18,480 keys.
     Returns (flops, seconds, threads)."""
     import numpy as np
     import torch
@@ -139,9 +139,9 @@ def oracle_sample(seconds_hint=True):
     from same_step_kv_b200 import synth
     q, k, v = synth.chunk_qkv(0, CHUNK, STEP, 0, T, HEADS, D)
     kf, vf = synth.store_fill(0, 0, STEP, HEADS, N_KEYS, D)
-    q, k, v = (t.double().numpy() for t in (q, k, v))
-    K = kf.double().numpy().transpose(1, 0, 2).copy()
-    V = vf.double().numpy().transpose(1, 0, 2).copy()
+    q, k, v = (t[:, :heads].double().numpy() for t in (q, k, v))
+    K = kf[:heads].double().numpy().transpose(1, 0, 2).copy()
+    V = vf[:heads].double().numpy().transpose(1, 0, 2).copy()
     t0 = time.perf_counter()
     f, hh, ww = rope.token_coords(T, W, HH, 2 + CHUNK)
     qr = rope.rotate(q, f, hh, ww)
@@ -151,7 +151,7 @@ def oracle_sample(seconds_hint=True):
     V[3 * T + slot * T: 3 * T + slot * T + T] = v
     attention.attend_heads(qr, K, V)
     dt = time.perf_counter() - t0
-    return ATTN_FLOPS, dt, torch.get_num_threads()
+    return ATTN_FLOPS * heads // HEADS, dt, torch.get_num_threads()
 
 
 def run_reference(args, rank):
@@ -159,7 +159,7 @@ def run_reference(args, rank):
         return
     vals = []
     for i in range(args.warmup + args.steps):
-        fl, dt, thr = oracle_sample()
+        fl, dt, thr = oracle_sample(heads=2)
         if i >= args.warmup:
             vals.append(fl / dt / 1e12)
     v = statistics.median(vals)
@@ -167,9 +167,10 @@ def run_reference(args, rank):
         "impl": "reference", "metric": "chunk-attention TFLOP/s", "value": v,
         "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": "one layer: RoPE + 880x18480 attention x 24 heads"},
+        "config": {"workload": WORKLOAD,
+                   "sample": "per step: RoPE + 880 x 18480 attention of 2 of the 24 heads of one layer"},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                         "sample": "one of the 30 layers per step (880 queries x 24 heads x 18480 keys)"},
+                         "sample": "per step: 2 heads of one layer (880 queries x 18480 keys each)"},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "vs_baseline": None,
     }
@@ -179,16 +180,19 @@ def run_reference(args, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="layers per step (30 in the profile; fewer only for small ncu captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.warmup < 3:
         args.warmup = 3
+    NL = args.layers
     if args.impl == "reference":
         run_reference(args, rank)
         return
@@ -205,19 +209,19 @@ def main():
     cs = torch.cuda.current_stream()
 
     # ---- setup: store with every layer's history at the steady state
-    cfg = pv.make_config(LAYERS, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
+    cfg = pv.make_config(NL, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
     store = pv.KVStore(cfg, device=dev)
     h = store.handle
     st = pv.pv_kv_state()
     st.phase, st.chunk = pv.PV_PHASE_STEADY, CHUNK
     pv.pv_kv_set_state(h, 0, st)
     Kr, Vr = store.k_region(), store.v_region()
-    for layer in range(LAYERS):
+    for layer in range(NL):
         kf, vf = synth.store_fill(rank, layer, STEP, HEADS, N_KEYS, D, dev)
         Kr[layer, STEP, 0] = kf
         Vr[layer, STEP, 0] = vf
     del kf, vf
-    qkv = [synth.chunk_qkv(rank, CHUNK, STEP, layer, T, HEADS, D, dev) for layer in range(LAYERS)]
+    qkv = [synth.chunk_qkv(rank, CHUNK, STEP, layer, T, HEADS, D, dev) for layer in range(NL)]
     q_rot = torch.empty(HEADS * T * D, dtype=torch.bfloat16, device=dev)
     out = torch.empty(T, HEADS, D, dtype=torch.bfloat16, device=dev)
     x = synth.latent(rank, 1, 48, 44, 80, dev).reshape(-1)
@@ -227,7 +231,7 @@ def main():
     attn_ev = []
 
     def step(record=False):
-        for layer in range(LAYERS):
+        for layer in range(NL):
             q, k, v = qkv[layer]
             pv.pv_rope_append(h, [0], layer, STEP, q, k, v, q_rot, cs)
             if record:
@@ -265,7 +269,7 @@ def main():
     ms_step = ms / args.steps
 
     # ---- e2e: the same step through the public API from pinned host buffers
-    hq = [tuple(t.cpu().pin_memory() for t in qkv[l]) for l in range(LAYERS)]
+    hq = [tuple(t.cpu().pin_memory() for t in qkv[l]) for l in range(NL)]
     hv = vel.cpu().pin_memory()
     hx = x.cpu().pin_memory()
     hres = torch.empty(LATENT, dtype=torch.float32).pin_memory()
@@ -278,7 +282,7 @@ def main():
     def e2e_step():
         with torch.cuda.stream(copy_s):
             dv.copy_(hv, non_blocking=True)
-        for layer in range(LAYERS):
+        for layer in range(NL):
             b = layer % 2
             with torch.cuda.stream(copy_s):
                 if layer >= 2:
@@ -309,18 +313,20 @@ def main():
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e2e_ms = float(tt.item())
-    h2d = LAYERS * 3 * T * HEADS * D * 2 + LATENT * 4
+    h2d = NL * 3 * T * HEADS * D * 2 + LATENT * 4
     d2h = LATENT * 4
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fl, dt, thr = oracle_sample()
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": "one of the 30 layers of a step: RoPE + 880x18480 attention, 24 heads"}
+        runs = [oracle_sample() for _ in range(4)]
+        fl, dt = runs[0][0], statistics.median(r[1] for r in runs)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": runs[0][2], "kind": "oracle",
+               "sample": "one of the 30 layers of a step (RoPE + 880 x 18480 attention, "
+                         "24 heads), median of 4 runs"}
 
     if rank == 0:
         peaks, src = load_peaks()
-        step_flops = LAYERS * ATTN_FLOPS * world
+        step_flops = NL * ATTN_FLOPS * world
         value = step_flops / (ms_step * 1e-3) / 1e12
         achieved = ATTN_FLOPS / (attn_ms * 1e-3) / 1e12
         peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
@@ -329,8 +335,8 @@ def main():
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "heads": HEADS, "head_dim": D, "queries": T,
-                       "keys": N_KEYS, "layers": LAYERS,
+            "config": {"workload": WORKLOAD if NL == LAYERS else WORKLOAD.replace("30 layers", f"{NL} layers"), "heads": HEADS, "head_dim": D, "queries": T,
+                       "keys": N_KEYS, "layers": NL,
                        "l2": "inputs larger than L2 (6.9 GB of K/V per step), no flush"},
             "latent_frames_per_s": world / (ms_step * 1e-3),
             "pct_of_bf16_peak": 100.0 * value / peak,
@@ -342,7 +348,7 @@ def main():
                          "ms_per_launch": attn_ms, "traffic": profiled_traffic()},
             "e2e": {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * (2 * LAYERS + 1),
+            "gpu_launches": args.steps * (2 * NL + 1),
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
