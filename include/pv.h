@@ -209,6 +209,26 @@ PV_API pv_status pv_attn_dense(const void* q, const void* k, const void* v, int 
                         int heads, int head_dim, void* out, float* lse, void* ws,
                         size_t ws_bytes, void* cuda_stream);
 
+/* Dense attention like pv_attn_dense (same layouts, same kernel), for
+ * callers that cannot allocate device memory where they call it: code inside
+ * a custom allocator or memory-pool callback, plugins whose host framework
+ * owns all device allocations, latency-critical paths that must not touch
+ * the allocator.  It takes no workspace and calls no allocating routine:
+ * its split-KV scratch is a fixed 8 MiB array inside the library, held by
+ * every GPU that loads the library until the process exits.  The pages
+ * describe no counterpart of this call; it is a property of this library.
+ *  - Limit: heads * ceil(n_q / 256) * 2 <= 16384 query tiles, else
+ *    PV_ERR_CAPACITY with a message naming the limit (use pv_attn_dense).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and clears the part it needs on
+ *    cuda_stream; calls whose executions overlap on the GPU (other streams,
+ *    other host threads) race on it and must be serialised by the caller. */
+PV_API pv_status pv_attn_dense_noalloc(const void* q, const void* k, const void* v, int n_q,
+                                       int n_k, int heads, int head_dim, void* out, float* lse,
+                                       void* cuda_stream);
+
 /* Flow-matching Euler update in place (blog chapter 5, "UniPC"):
  *  x[i] += dsigma * v[i] for i < n, f32, one fused multiply-add per element.
  *  dsigma = sigma_next - sigma (negative while denoising), computed by the

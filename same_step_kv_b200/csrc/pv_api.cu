@@ -146,6 +146,8 @@ pv_status check_device(int* n_sm) {
 
 namespace pv {
 
+pv_status report_error(pv_status code, const char* msg) { return fail(code, "%s", msg); }
+
 bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, char* err,
                      size_t errlen) {
     auto enc = get_encode();

@@ -92,6 +92,9 @@ cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaS
 bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, char* err,
                      size_t errlen);
 
+// Records a failure for pv_last_error() and returns code.
+pv_status report_error(pv_status code, const char* msg);
+
 // Split-KV plan for one attention launch: fills n_split, unit0, part0, cnt0.
 // Returns the number of CTAs, or -1 when the partial slots do not suffice.
 int plan_attention(AttnStreamDesc* st, int n_streams, int heads, int n_sm, int part_capacity,

@@ -74,6 +74,7 @@ _SIGS = {
     "pv_rope_dense": ([_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "pv_attn_dense_ws_bytes": ([_i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "pv_attn_dense": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
+    "pv_attn_dense_noalloc": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp], _i),
     "pv_euler_step": ([_vp, _vp, _sz, ctypes.c_float, _vp], _i),
     "pv_kv_poll_device_error": ([_vp, ctypes.POINTER(_i)], _i),
 }
@@ -202,6 +203,12 @@ def pv_attn_dense(q, k, v, n_q, n_k, heads, head_dim, out, lse, ws, ws_bytes,
                   cuda_stream=None) -> None:
     _check(lib.pv_attn_dense(_ptr(q), _ptr(k), _ptr(v), n_q, n_k, heads, head_dim, _ptr(out),
                              _ptr(lse), _ptr(ws), ws_bytes, _stream(cuda_stream)))
+
+
+def pv_attn_dense_noalloc(q, k, v, n_q, n_k, heads, head_dim, out, lse=None,
+                          cuda_stream=None) -> None:
+    _check(lib.pv_attn_dense_noalloc(_ptr(q), _ptr(k), _ptr(v), n_q, n_k, heads, head_dim,
+                                     _ptr(out), _ptr(lse), _stream(cuda_stream)))
 
 
 def pv_euler_step(x, v, n, dsigma, cuda_stream=None) -> None:
