@@ -235,6 +235,13 @@ PV_API pv_status pv_attn_dense_noalloc(const void* q, const void* k, const void*
  *  caller in fp64 and passed rounded to f32. */
 PV_API pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* cuda_stream);
 
+/* Self-test of the attention kernel's software exponential: y[i] = 2^x[i]
+ * computed as that kernel computes a quarter of its softmax exponentials
+ * (round-to-nearest range reduction and a fitted minimax cubic; maximum
+ * relative error 7.5e-5 for x in [-125, 128)).  x, y: f32 device arrays of n
+ * elements.  Used by the tests to compare against exp2. */
+PV_API pv_status pv_selftest_exp2_poly(const float* x, float* y, size_t n, void* cuda_stream);
+
 /* Reads (synchronously) and clears the device error word that the kernels of
  * this handle set when a bounded device-side wait gives up.  *code is 0 when
  * no wait timed out. */

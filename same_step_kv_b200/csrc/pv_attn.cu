@@ -107,6 +107,44 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Bars* b
     return true;
 }
 
+#ifndef PV_MMA_SPIN
+#define PV_MMA_SPIN 1
+#endif
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait that never suspends the thread: for the single MMA-issuing
+// thread, whose reaction time is on the critical path of every tile.
+__device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, Bars* b, int* err) {
+#if PV_MMA_SPIN
+    if (mbar_test(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 255) == 0) {
+            if (*(volatile int*)&b->abort) return false;
+            if (clock64() - t0 > kWaitCycles) {
+                atomicExch(err, 1);
+                *(volatile int*)&b->abort = 1;
+                return false;
+            }
+        }
+    }
+#else
+    return mbar_wait(bar, parity, b, err);
+#endif
+}
+
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
                                          uint32_t bar) {
@@ -209,6 +247,12 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -325,7 +369,7 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
             mma_ts(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
                    (acc || kk > 0) ? 1u : 0u);
     };
-    bool ok = mbar_wait(smem_u32(&b->q_full), 0, b, p.err);
+    bool ok = mbar_spin(smem_u32(&b->q_full), 0, b, p.err);
     tc_fence_after();
     const int n = u.n_iter;
     for (int j = 0; ok && j < n; ++j) {
@@ -334,19 +378,19 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
         const int vs_prev = (2 * j - 1 + C::kStages) % C::kStages;
         const uint32_t vph_prev = ((2 * j - 1) / C::kStages) & 1;
         if (j > 0) {
-            ok = mbar_wait(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
-                 mbar_wait(smem_u32(&b->p_full[0]), (j - 1) & 1, b, p.err);
+            ok = mbar_spin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
+                 mbar_spin(smem_u32(&b->p_full[0]), (j - 1) & 1, b, p.err);
             if (!ok) break;
             tc_fence_after();
             pv(0, vs_prev, j > 1);
         }
-        if (!(ok = mbar_wait(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
+        if (!(ok = mbar_spin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
         tc_fence_after();
         qk(0, ks);
         tc_commit(smem_u32(&b->s_full[0]));
         if (hasB) {
             if (j > 0) {
-                if (!(ok = mbar_wait(smem_u32(&b->p_full[1]), (j - 1) & 1, b, p.err))) break;
+                if (!(ok = mbar_spin(smem_u32(&b->p_full[1]), (j - 1) & 1, b, p.err))) break;
                 tc_fence_after();
                 pv(1, vs_prev, j > 1);
             }
@@ -359,13 +403,13 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
     if (ok) {
         const int vs = (2 * n - 1) % C::kStages;
         const uint32_t vph = ((2 * n - 1) / C::kStages) & 1;
-        ok = mbar_wait(smem_u32(&b->kv_full[vs]), vph, b, p.err) &&
-             mbar_wait(smem_u32(&b->p_full[0]), (n - 1) & 1, b, p.err);
+        ok = mbar_spin(smem_u32(&b->kv_full[vs]), vph, b, p.err) &&
+             mbar_spin(smem_u32(&b->p_full[0]), (n - 1) & 1, b, p.err);
         if (ok) {
             tc_fence_after();
             pv(0, vs, n > 1);
             tc_commit(smem_u32(&b->o_full[0]));
-            if (hasB && (ok = mbar_wait(smem_u32(&b->p_full[1]), (n - 1) & 1, b, p.err))) {
+            if (hasB && (ok = mbar_spin(smem_u32(&b->p_full[1]), (n - 1) & 1, b, p.err))) {
                 tc_fence_after();
                 pv(1, vs, n > 1);
                 tc_commit(smem_u32(&b->o_full[1]));
@@ -380,6 +424,40 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
     }
 }
 
+// One pass of exponentials over this thread's 128 scores: p = 2^(s*sl2 - m)
+// on the XU pipe, written to TMEM as bf16 pairs over the first 64 columns of
+// S.  The bf16 value is the upper half of the f32 (round toward zero, a
+// byte permute on the ALU pipe instead of a conversion on the XU pipe), and
+// the row sum accumulates exactly those rounded values, so that P and its
+// normaliser agree.  Returns max(s*sl2 - m) over the row (masked: -inf).
+__device__ __forceinline__ float exp_pass(const uint32_t* sr, float sl2, float m, uint32_t tS,
+                                          float& l_tile) {
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    const float2 nmx2 = make_float2(-m, -m);
+    float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+    float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 128; c += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sr[c + i]), __uint_as_float(sr[c + i + 1])), sl2x2,
+                nmx2);
+            xm[(i >> 1) & 3] = fmax3(xm[(i >> 1) & 3], x.x, x.y);
+            const uint32_t b0 = __float_as_uint(ex2(x.x)) & 0xFFFF0000u;
+            const uint32_t b1 = __float_as_uint(ex2(x.y)) & 0xFFFF0000u;
+            acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3],
+                                           make_float2(__uint_as_float(b0), __uint_as_float(b1)));
+            pk[i / 2] = __byte_perm(b0, b1, 0x7632);
+        }
+        tmem_st16(tS + c / 2, pk);
+    }
+    const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+    l_tile = a.x + a.y;
+    return fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
+}
+
 template <int D>
 __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, uint32_t tmem,
                                  int X) {
@@ -392,7 +470,8 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
     const uint32_t tO = tmem + lane + C::kColsO + X * D;
     const float sl2 = p.scale_log2;
     float m = -INFINITY;  // maximum applied to the exponentials, log2 units
-    float l = 0.f;        // sum of the exponentials
+    float l = 0.f;        // sum of the exponentials (as rounded into P)
+    float l_tile = 0.f;
     bool ok = true;
     for (int j = 0; j < u.n_iter; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->s_full[X]), j & 1, b, p.err));
@@ -406,18 +485,29 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
             for (int c = 0; c < 128; ++c)
                 if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(sr[0]);
+        if (j == 0) {
+            // first tile: the running maximum starts from this tile's maximum
+            float mx8[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-        const float m_new = fmaxf(m, mx * sl2);
-        const bool need = m_new > m + 8.0f;
-        // tcgen05.ld / st are warp-collective: rescale when any lane needs it
-        if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? ex2(m - m_new) : 1.0f;  // 0 on the first tile
-            if (need) {
-                l *= alpha;
-                m = m_new;
-            }
+            for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+#pragma unroll
+            for (int c = 8; c < 128; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mx8[i] = fmax3(mx8[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+            m = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                      fmaxf(mx8[6], mx8[7])) * sl2;
+        }
+        // Exponentials with the maximum in hand; the tile's own maximum is
+        // tracked alongside, off the critical path.  Only if some score rose
+        // more than 8 (log2 units) above m is the tile redone with a larger m.
+        float xmax = exp_pass(sr, sl2, m, tS, l_tile);
+        if (__any_sync(0xffffffffu, xmax > 8.0f)) {
+            const bool need = xmax > 8.0f;
+            const float m_new = need ? m + xmax : m;
+            const float alpha = ex2(m - m_new);
+            l *= alpha;
+            m = m_new;
             if (j > 0) {
                 // O holds P V of tiles < j, complete: S(j) was committed after it
 #pragma unroll 1
@@ -430,25 +520,13 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
                     tmem_st32(tO + c, o);
                 }
             }
+            exp_pass(sr, sl2, m, tS, l_tile);
         }
-        float sum = 0.f;
-        const float nm = -m;
-#pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[c + i]), sl2, nm));
-                const float p1 = ex2(fmaf(__uint_as_float(sr[c + i + 1]), sl2, nm));
-                sum += p0 + p1;
-                pk[i / 2] = pack_bf16(p0, p1);
-            }
-            tmem_st16(tS + c / 2, pk);
-        }
-        l += sum;
+        l += l_tile;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&b->p_full[X]));
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->p_full[X]));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->o_full[X]), 0, b, p.err));
     if (ok) tc_fence_after();
@@ -483,7 +561,9 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
         return;
     }
 
-    // split-KV: store the unnormalised partial, the last of the parts merges
+    // split-KV: store the unnormalised partial, the last of the parts merges.
+    // A slot is column-major ([D][128] then m[128], l[128]) so that the 32
+    // lanes of a warp always touch 32 consecutive floats.
     const size_t slot_f = partial_slot_floats(D);
     const int tile_id = (u.head * s.n_qb + u.qb) * kQTilesPerCta + X;
     const size_t slot0 = (size_t)s.part0 + (size_t)tile_id * s.n_split;
@@ -491,20 +571,15 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
 #pragma unroll 1
     for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
+        if (ok) tmem_ld32_wait(tO + c, o);
         if (ok) {
-            tmem_ld32_wait(tO + c, o);
-        }
-        if (row_ok) {
-            float4* d4 = reinterpret_cast<float4*>(mine + (size_t)r * D + c);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                    __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            for (int i = 0; i < 32; ++i) __stcg(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]));
         }
     }
-    if (row_ok) {
-        mine[(size_t)kQRows * D + r] = m;
-        mine[(size_t)kQRows * D + kQRows + r] = l;
+    if (ok) {
+        __stcg(mine + (size_t)kQRows * D + r, m);
+        __stcg(mine + (size_t)kQRows * D + kQRows + r, l);
     }
     __threadfence();
     named_sync(1 + X, 128);
@@ -532,25 +607,24 @@ __device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, ui
     const float invL = 1.0f / L;
     bf16* dst = p.out + ((size_t)tok * p.heads + u.head) * D;
 #pragma unroll 1
-    for (int c = 0; c < D; c += 8) {
-        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int c = 0; c < D; c += 16) {
+        float acc[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc[k] = 0.f;
         for (int i = 0; i < s.n_split; ++i) {
             const float* pi = p.partial + (slot0 + i) * slot_f;
             const float w = ex2(__ldcg(pi + (size_t)kQRows * D + r) - M) * invL;
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(pi + (size_t)r * D + c));
-            const float4 bq = __ldcg(reinterpret_cast<const float4*>(pi + (size_t)r * D + c + 4));
-            acc[0] = fmaf(w, a.x, acc[0]);
-            acc[1] = fmaf(w, a.y, acc[1]);
-            acc[2] = fmaf(w, a.z, acc[2]);
-            acc[3] = fmaf(w, a.w, acc[3]);
-            acc[4] = fmaf(w, bq.x, acc[4]);
-            acc[5] = fmaf(w, bq.y, acc[5]);
-            acc[6] = fmaf(w, bq.z, acc[6]);
-            acc[7] = fmaf(w, bq.w, acc[7]);
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = __ldcg(pi + (size_t)(c + k) * kQRows + r);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[k] = fmaf(w, v[k], acc[k]);
         }
-        *reinterpret_cast<uint4*>(dst + c) =
-            make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
-                       pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+        d4[0] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                           pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+        d4[1] = make_uint4(pack_bf16(acc[8], acc[9]), pack_bf16(acc[10], acc[11]),
+                           pack_bf16(acc[12], acc[13]), pack_bf16(acc[14], acc[15]));
     }
     if (p.lse) p.lse[(size_t)tok * p.heads + u.head] = (M + __log2f(L)) * ln2;
 }
@@ -572,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&b->q_full), 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&b->s_full[x]), 1);
-            mbar_init(smem_u32(&b->p_full[x]), 128);
+            mbar_init(smem_u32(&b->p_full[x]), 4);  // one arrive per softmax warp
             mbar_init(smem_u32(&b->o_full[x]), 1);
         }
         mbar_init(smem_u32(&b->mma_done), 1);

@@ -12,7 +12,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpv.so")
+# PV_LIB may name another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("PV_LIB") or os.path.join(_HERE, "libpv.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is not built; run `python -m same_step_kv_b200.build`")
 lib = ctypes.CDLL(LIB_PATH)
@@ -77,6 +78,7 @@ _SIGS = {
     "pv_attn_dense_noalloc": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp], _i),
     "pv_euler_step": ([_vp, _vp, _sz, ctypes.c_float, _vp], _i),
     "pv_kv_poll_device_error": ([_vp, ctypes.POINTER(_i)], _i),
+    "pv_selftest_exp2_poly": ([_vp, _vp, _sz, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -219,6 +221,10 @@ def pv_kv_poll_device_error(kv) -> int:
     c = _i()
     _check(lib.pv_kv_poll_device_error(kv, ctypes.byref(c)))
     return c.value
+
+
+def pv_selftest_exp2_poly(x, y, n, cuda_stream=None) -> None:
+    _check(lib.pv_selftest_exp2_poly(_ptr(x), _ptr(y), n, _stream(cuda_stream)))
 
 
 # ------------------------------------------------------------------ helpers
