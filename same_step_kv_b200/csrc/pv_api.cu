@@ -69,9 +69,8 @@ WsLayout ws_layout(const pv_kv_config& c) {
     const int max_q = c.first_frames * T;
     const int n_qb = (max_q + kQBlock - 1) / kQBlock;
     w.n_counters = c.max_streams * c.heads * n_qb * kQTilesPerCta;
-    // Enough partial slots that every query tile of the largest launch may be
-    // split 8 ways, capped so that small configurations stay small.
-    w.n_partials = std::min(w.n_counters * 8, 8192);
+    // Stream-K partial results: 4 slots per CTA, at most kMaxGrid CTAs.
+    w.n_partials = 4 * kMaxGrid;
     w.n_table = c.max_frames * c.rope_pairs_t + c.frame_h * c.rope_pairs_h +
                 c.frame_w * c.rope_pairs_w;
     w.err_off = 0;
@@ -584,13 +583,11 @@ pv_status pv_chunk_attn(pv_kv kv, int n_streams, const int* streams, int layer, 
         a.out_tok0 = tok;
         tok += d.n_queries;
     }
-    int order[PV_MAX_STREAMS];
-    const int units = plan_attention(p.st, n_streams, c.heads, kv->n_sm, kv->wl.n_partials,
-                                     kv->wl.n_counters, order);
-    if (units < 0) return fail(PV_ERR_CAPACITY, "split-KV plan exceeds the workspace");
+    if (plan_attention(p, kv->n_sm, kv->wl.n_partials, kv->wl.n_counters) < 0)
+        return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
     CUtensorMap tq;
     if ((st = q_map(kv, q_rot, (long long)c.heads * tok, &tq))) return st;
-    cudaError_t e = launch_attn(tq, kv->tm_k, kv->tm_v, p, units, (cudaStream_t)cuda_stream);
+    cudaError_t e = launch_attn(tq, kv->tm_k, kv->tm_v, p, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "chunk_attn launch");
     return PV_OK;
 }
@@ -649,7 +646,8 @@ pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_dim, size
         return fail(PV_ERR_SHAPE, "bad dense attention shape");
     const size_t n_qb = (n_q + kQBlock - 1) / kQBlock;
     const size_t n_cnt = (size_t)heads * n_qb * kQTilesPerCta;
-    const size_t n_part = std::min<size_t>(n_cnt * 8, 8192);
+    const size_t tiles = (size_t)heads * n_qb * ((n_k + kKeyTile - 1) / kKeyTile);
+    const size_t n_part = 4 * std::min<size_t>(kMaxGrid, tiles);
     *ws_bytes = 256 + round_up(n_cnt * sizeof(int), 256) +
                 n_part * partial_slot_floats(head_dim) * sizeof(float);
     return PV_OK;
@@ -676,7 +674,8 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
     if ((st = check_device(&n_sm))) return st;
     const size_t n_qb = (n_q + kQBlock - 1) / kQBlock;
     const int n_cnt = (int)((size_t)heads * n_qb * kQTilesPerCta);
-    const int n_part = (int)std::min<size_t>((size_t)n_cnt * 8, 8192);
+    const size_t tiles = (size_t)heads * n_qb * ((n_k + kKeyTile - 1) / kKeyTile);
+    const int n_part = (int)(4 * std::min<size_t>(kMaxGrid, tiles));
     AttnParams p{};
     p.out = (bf16*)out;
     p.lse = lse;
@@ -694,16 +693,15 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
     a.kv_row0 = 0;
     a.kv_head_stride = n_k;
     a.out_tok0 = 0;
-    int order[1];
-    const int units = plan_attention(p.st, 1, heads, n_sm, n_part, n_cnt, order);
-    if (units < 0) return fail(PV_ERR_CAPACITY, "split-KV plan exceeds the workspace");
+    if (plan_attention(p, n_sm, n_part, n_cnt) < 0)
+        return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
     CUtensorMap tq, tk, tv;
     char msg[256];
     if (!encode_rows_map(&tq, q, (long long)heads * n_q, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tk, k, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg))
         return fail(PV_ERR_CUDA, "%s", msg);
-    cudaError_t e = launch_attn(tq, tk, tv, p, units, (cudaStream_t)cuda_stream);
+    cudaError_t e = launch_attn(tq, tk, tv, p, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_dense launch");
     return PV_OK;
 }

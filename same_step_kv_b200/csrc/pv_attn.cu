@@ -35,8 +35,8 @@ namespace pv {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kRegsLow = 80;    // warpgroup 0 after setmaxnreg.dec
-constexpr int kRegsHigh = 208;  // softmax warpgroups after setmaxnreg.inc
+constexpr int kRegsLow = 96;    // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsHigh = 200;  // softmax warpgroups after setmaxnreg.inc
 static_assert(kRegsLow * 128 + 2 * kRegsHigh * 128 <= 168 * kThreads, "register split");
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 
@@ -48,12 +48,16 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    static constexpr int kSmem = kBarOff + 256 + 1024;       // + barriers + alignment slack
+    static constexpr int kSmem = kBarOff + 512 + 1024;       // + barriers + alignment slack
     static constexpr uint32_t kColsO = 256;
 };
 
-struct Bars {
+struct Bars {  // 264 bytes, inside the 512 reserved after the tiles
     uint64_t q_full;
+    uint64_t q_empty;
+    uint64_t o_empty[2];
+    uint64_t ep_in[2];    // split epilogue: the 4 softmax warps of a tile wrote their partial
+    uint64_t ep_out[2];   // split epilogue: the arrival count is in last[]
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_full[2];
@@ -264,90 +268,132 @@ __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-struct Unit {
-    int si, head, qb, split, kt0, n_iter, q0, rows[2];
+// ----------------------------------------------------------------- schedule
+// CTA c owns the key tiles [bound(c), bound(c+1)) of the launch's item list
+// (see pv_plan.cu).  A segment is the part of one item inside that range.
+__device__ __forceinline__ long long bound(const AttnParams& p, int c) {
+    if (!p.item_aligned) return (long long)c * p.total / p.grid;
+    // whole items: CTA c starts at item c * n_items / grid
+    const int k = (int)((long long)c * p.n_items / p.grid);
+    int i = 0;
+    while (i + 1 < p.n_streams && p.st[i + 1].item0 <= k) ++i;
+    if (k >= p.n_items) return p.total;
+    return p.st[i].cost0 + (long long)(k - p.st[i].item0) * p.st[i].n_kt;
+}
+// The CTA whose range holds key tile x.
+__device__ __forceinline__ int cta_of(const AttnParams& p, long long x) {
+    return (int)(((x + 1) * p.grid - 1) / p.total);
+}
+
+struct Seg {
+    int si, head, qb, kt0, n, q0, rows[2];
+    int item;      // global item index
+    int c_first;   // first CTA holding part of the item
+    int nseg;      // CTAs holding parts of the item
+    int which;     // 0: this CTA's first segment, 1: a later one
 };
 
-__device__ __forceinline__ Unit decode_unit(const AttnParams& p) {
-    Unit u{};
-    const int b = blockIdx.x;
-    for (int i = 0; i < p.n_streams; ++i) {
+struct SegIter {
+    long long pos, end;
+    __device__ SegIter(const AttnParams& p) : pos(bound(p, blockIdx.x)), end(bound(p, blockIdx.x + 1)) {}
+    __device__ bool next(const AttnParams& p, Seg& g) {
+        if (pos >= end) return false;
+        int i = 0;
+        while (i + 1 < p.n_streams && p.st[i + 1].cost0 <= pos) ++i;
         const AttnStreamDesc& s = p.st[i];
-        const int n = p.heads * s.n_qb * s.n_split;
-        if (b >= s.unit0 && b < s.unit0 + n) {
-            u.si = i;
-            int r = b - s.unit0;
-            u.split = r % s.n_split;
-            r /= s.n_split;
-            u.qb = r % s.n_qb;
-            u.head = r / s.n_qb;
-            u.kt0 = (int)((long long)u.split * s.n_kt / s.n_split);
-            u.n_iter = (int)((long long)(u.split + 1) * s.n_kt / s.n_split) - u.kt0;
-            u.q0 = u.qb * kQBlock;
-            u.rows[0] = min(kQRows, s.n_q - u.q0);
-            u.rows[1] = max(0, min(kQRows, s.n_q - u.q0 - kQRows));
-            return u;
+        const long long off = pos - s.cost0;
+        const int li = (int)(off / s.n_kt);
+        g.si = i;
+        g.kt0 = (int)(off - (long long)li * s.n_kt);
+        const long long i0 = s.cost0 + (long long)li * s.n_kt;   // the item's key-tile range
+        const long long i1 = i0 + s.n_kt;
+        const long long e = i1 < end ? i1 : end;
+        g.n = (int)(e - pos);
+        g.which = pos == bound(p, blockIdx.x) ? 0 : 1;
+        g.head = li / s.n_qb;
+        g.qb = li - g.head * s.n_qb;
+        g.item = s.item0 + li;
+        if (p.item_aligned) {
+            g.c_first = blockIdx.x;
+            g.nseg = 1;
+        } else {
+            g.c_first = cta_of(p, i0);
+            g.nseg = cta_of(p, i1 - 1) - g.c_first + 1;
         }
+        g.q0 = g.qb * kQBlock;
+        g.rows[0] = min(kQRows, s.n_q - g.q0);
+        g.rows[1] = max(0, min(kQRows, s.n_q - g.q0 - kQRows));
+        pos = e;
+        return true;
     }
-    u.si = -1;
-    return u;
+};
+
+// Partial slot of CTA c's part of an item starting at key tile i0, tile X.
+__device__ __forceinline__ size_t part_slot(const AttnParams& p, int c, long long i0, int X) {
+    const int which = i0 <= bound(p, c) ? 0 : 1;
+    return ((size_t)c * 2 + which) * 2 + X;
 }
 
 // ----------------------------------------------------------------- roles
 template <int D>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                         const AttnParams& p, const Unit& u, uint8_t* smem, Bars* b) {
+                         const AttnParams& p, uint8_t* smem, Bars* b) {
     using C = Cfg<D>;
-    const AttnStreamDesc& s = p.st[u.si];
-    const int ntile = u.rows[1] > 0 ? 2 : 1;
     const uint32_t qbar = smem_u32(&b->q_full);
-    mbar_expect_tx(qbar, ntile * C::kTileBytes);
-    const int qrow = s.q_row0 + u.head * s.n_q + u.q0;
-    for (int t = 0; t < ntile; ++t)
-        for (int c = 0; c < C::kSub; ++c)
-            tma_load(smem_u32(smem + C::kQOff + t * C::kTileBytes + c * 16384), tq, c * 64,
-                     qrow + t * kQRows, qbar);
-    const int krow0 = s.kv_row0 + u.head * s.kv_head_stride + u.kt0 * kKeyTile;
-    int issued = 0;
-    for (int j = 0; j < u.n_iter && !b->abort; ++j) {
-        for (int w = 0; w < 2; ++w) {
-            const int idx = 2 * j + w;
-            const int st = idx % C::kStages;
-            const uint32_t ph = (idx / C::kStages) & 1;
-            if (!mbar_wait(smem_u32(&b->kv_empty[st]), ph ^ 1, b, p.err)) break;
-            const uint32_t full = smem_u32(&b->kv_full[st]);
-            mbar_expect_tx(full, C::kTileBytes);
-            const CUtensorMap* m = w == 0 ? tk : tv;
+    int kv = 0, qseg = 0;
+    bool ok = true;
+    SegIter it(p);
+    Seg g;
+    while (ok && it.next(p, g)) {
+        const AttnStreamDesc& s = p.st[g.si];
+        const int ntile = g.rows[1] > 0 ? 2 : 1;
+        // the previous segment's S products are done with the Q tiles
+        if (!(ok = mbar_wait(smem_u32(&b->q_empty), (qseg & 1) ^ 1, b, p.err))) break;
+        mbar_expect_tx(qbar, ntile * C::kTileBytes);
+        const int qrow = s.q_row0 + g.head * s.n_q + g.q0;
+        for (int t = 0; t < ntile; ++t)
             for (int c = 0; c < C::kSub; ++c)
-                tma_load(smem_u32(smem + C::kKVOff + st * C::kTileBytes + c * 16384), m, c * 64,
-                         krow0 + j * kKeyTile, full);
-            issued = idx + 1;
+                tma_load(smem_u32(smem + C::kQOff + t * C::kTileBytes + c * 16384), tq, c * 64,
+                         qrow + t * kQRows, qbar);
+        ++qseg;
+        const int krow0 = s.kv_row0 + g.head * s.kv_head_stride + g.kt0 * kKeyTile;
+        for (int j = 0; ok && j < g.n; ++j) {
+            for (int w = 0; w < 2; ++w) {
+                const int st = kv % C::kStages;
+                const uint32_t ph = (kv / C::kStages) & 1;
+                if (!(ok = mbar_wait(smem_u32(&b->kv_empty[st]), ph ^ 1, b, p.err))) break;
+                const uint32_t full = smem_u32(&b->kv_full[st]);
+                mbar_expect_tx(full, C::kTileBytes);
+                const CUtensorMap* m = w == 0 ? tk : tv;
+                for (int c = 0; c < C::kSub; ++c)
+                    tma_load(smem_u32(smem + C::kKVOff + st * C::kTileBytes + c * 16384), m,
+                             c * 64, krow0 + j * kKeyTile, full);
+                ++kv;
+            }
         }
     }
     // Before leaving, make sure no copy of ours is still landing in shared
-    // memory: wait (bounded) for the last load issued into each stage.
-    for (int idx = max(0, issued - C::kStages); idx < issued; ++idx) {
-        const int st = idx % C::kStages;
+    // memory: wait (bounded) for the last load issued into each stage, and
+    // for the last Q load.
+    for (int idx = max(0, kv - C::kStages); idx < kv; ++idx) {
+        const uint32_t bar = smem_u32(&b->kv_full[idx % C::kStages]);
         const uint32_t ph = (idx / C::kStages) & 1;
-        const uint32_t bar = smem_u32(&b->kv_full[st]);
         const long long t0 = clock64();
         while (!mbar_try(bar, ph) && clock64() - t0 < kWaitCycles) {
         }
     }
-    {
+    if (qseg > 0) {
         const long long t0 = clock64();
-        while (!mbar_try(qbar, 0) && clock64() - t0 < kWaitCycles) {
+        while (!mbar_try(qbar, (qseg - 1) & 1) && clock64() - t0 < kWaitCycles) {
         }
     }
 }
 
 template <int D>
-__device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Bars* b,
-                           uint32_t tmem) {
+__device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t tmem) {
     using C = Cfg<D>;
     constexpr uint32_t idesc_qk = idesc_bf16(kQRows, kKeyTile, false);
     constexpr uint32_t idesc_pv = idesc_bf16(kQRows, D, true);
-    const bool hasB = u.rows[1] > 0;
     const uint32_t sQ = smem_u32(smem + C::kQOff);
     const uint32_t sKV = smem_u32(smem + C::kKVOff);
     auto qk = [&](int X, int stage) {
@@ -369,53 +415,66 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
             mma_ts(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
                    (acc || kk > 0) ? 1u : 0u);
     };
-    bool ok = mbar_spin(smem_u32(&b->q_full), 0, b, p.err);
-    tc_fence_after();
-    const int n = u.n_iter;
-    for (int j = 0; ok && j < n; ++j) {
-        const int ks = (2 * j) % C::kStages;
-        const uint32_t kph = ((2 * j) / C::kStages) & 1;
-        const int vs_prev = (2 * j - 1 + C::kStages) % C::kStages;
-        const uint32_t vph_prev = ((2 * j - 1) / C::kStages) & 1;
-        if (j > 0) {
-            ok = mbar_spin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
-                 mbar_spin(smem_u32(&b->p_full[0]), (j - 1) & 1, b, p.err);
-            if (!ok) break;
-            tc_fence_after();
-            pv(0, vs_prev, j > 1);
-        }
-        if (!(ok = mbar_spin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
+    int kv = 0, qseg = 0;
+    int pc[2] = {0, 0};  // P tiles consumed, per query tile
+    int oc[2] = {0, 0};  // segments finished, per query tile
+    bool ok = true;
+    // P V of tile X for key tile j of the current segment; the first one of
+    // a segment overwrites O, which the previous segment's epilogue must
+    // have read out first.
+    auto do_pv = [&](int X, int stage, int j) -> bool {
+        if (j == 0 && !mbar_spin(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
+        if (!mbar_spin(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
+        ++pc[X];
         tc_fence_after();
-        qk(0, ks);
-        tc_commit(smem_u32(&b->s_full[0]));
-        if (hasB) {
+        pv(X, stage, j > 0);
+        return true;
+    };
+    SegIter it(p);
+    Seg g;
+    while (ok && it.next(p, g)) {
+        const bool hasB = g.rows[1] > 0;
+        if (!(ok = mbar_spin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
+        ++qseg;
+        tc_fence_after();
+        const int n = g.n;
+        for (int j = 0; ok && j < n; ++j) {
+            const int ks = (kv + 2 * j) % C::kStages;
+            const uint32_t kph = ((kv + 2 * j) / C::kStages) & 1;
+            const int vs_prev = (kv + 2 * j - 1) % C::kStages;
+            const uint32_t vph_prev = ((kv + 2 * j - 1) / C::kStages) & 1;
             if (j > 0) {
-                if (!(ok = mbar_spin(smem_u32(&b->p_full[1]), (j - 1) & 1, b, p.err))) break;
-                tc_fence_after();
-                pv(1, vs_prev, j > 1);
+                if (!(ok = mbar_spin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
+                           do_pv(0, vs_prev, j - 1)))
+                    break;
             }
-            qk(1, ks);
-            tc_commit(smem_u32(&b->s_full[1]));
-        }
-        if (j > 0) tc_commit(smem_u32(&b->kv_empty[vs_prev]));
-        tc_commit(smem_u32(&b->kv_empty[ks]));
-    }
-    if (ok) {
-        const int vs = (2 * n - 1) % C::kStages;
-        const uint32_t vph = ((2 * n - 1) / C::kStages) & 1;
-        ok = mbar_spin(smem_u32(&b->kv_full[vs]), vph, b, p.err) &&
-             mbar_spin(smem_u32(&b->p_full[0]), (n - 1) & 1, b, p.err);
-        if (ok) {
+            if (!(ok = mbar_spin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
             tc_fence_after();
-            pv(0, vs, n > 1);
-            tc_commit(smem_u32(&b->o_full[0]));
-            if (hasB && (ok = mbar_spin(smem_u32(&b->p_full[1]), (n - 1) & 1, b, p.err))) {
-                tc_fence_after();
-                pv(1, vs, n > 1);
-                tc_commit(smem_u32(&b->o_full[1]));
+            qk(0, ks);
+            tc_commit(smem_u32(&b->s_full[0]));
+            if (hasB) {
+                if (j > 0 && !(ok = do_pv(1, vs_prev, j - 1))) break;
+                qk(1, ks);
+                tc_commit(smem_u32(&b->s_full[1]));
             }
-            tc_commit(smem_u32(&b->kv_empty[vs]));
+            if (j > 0) tc_commit(smem_u32(&b->kv_empty[vs_prev]));
+            tc_commit(smem_u32(&b->kv_empty[ks]));
         }
+        if (!ok) break;
+        tc_commit(smem_u32(&b->q_empty));  // the Q tiles are free once these S products end
+        const int vs = (kv + 2 * n - 1) % C::kStages;
+        const uint32_t vph = ((kv + 2 * n - 1) / C::kStages) & 1;
+        if (!(ok = mbar_spin(smem_u32(&b->kv_full[vs]), vph, b, p.err) && do_pv(0, vs, n - 1)))
+            break;
+        tc_commit(smem_u32(&b->o_full[0]));
+        ++oc[0];
+        if (hasB) {
+            if (!(ok = do_pv(1, vs, n - 1))) break;
+            tc_commit(smem_u32(&b->o_full[1]));
+            ++oc[1];
+        }
+        tc_commit(smem_u32(&b->kv_empty[vs]));
+        kv += 2 * n;
     }
     // every MMA issued by this thread has completed once mma_done flips
     tc_commit(smem_u32(&b->mma_done));
@@ -424,18 +483,20 @@ __device__ void mma_issuer(const AttnParams& p, const Unit& u, uint8_t* smem, Ba
     }
 }
 
+#ifndef PV_TRACK_MAX
+#define PV_TRACK_MAX 0
+#endif
 // One pass of exponentials over this thread's 128 scores: p = 2^(s*sl2 - m)
 // on the XU pipe, written to TMEM as bf16 pairs over the first 64 columns of
 // S.  The bf16 value is the upper half of the f32 (round toward zero, a
 // byte permute on the ALU pipe instead of a conversion on the XU pipe), and
 // the row sum accumulates exactly those rounded values, so that P and its
-// normaliser agree.  Returns max(s*sl2 - m) over the row (masked: -inf).
-__device__ __forceinline__ float exp_pass(const uint32_t* sr, float sl2, float m, uint32_t tS,
-                                          float& l_tile) {
+// normaliser agree.
+__device__ __forceinline__ void exp_pass(const uint32_t* sr, float sl2, float m, uint32_t tS,
+                                         float& l_tile) {
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 nmx2 = make_float2(-m, -m);
     float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-    float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int c = 0; c < 128; c += 32) {
         uint32_t pk[16];
@@ -444,7 +505,6 @@ __device__ __forceinline__ float exp_pass(const uint32_t* sr, float sl2, float m
             const float2 x = __ffma2_rn(
                 make_float2(__uint_as_float(sr[c + i]), __uint_as_float(sr[c + i + 1])), sl2x2,
                 nmx2);
-            xm[(i >> 1) & 3] = fmax3(xm[(i >> 1) & 3], x.x, x.y);
             const uint32_t b0 = __float_as_uint(ex2(x.x)) & 0xFFFF0000u;
             const uint32_t b1 = __float_as_uint(ex2(x.y)) & 0xFFFF0000u;
             acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3],
@@ -455,178 +515,197 @@ __device__ __forceinline__ float exp_pass(const uint32_t* sr, float sl2, float m
     }
     const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     l_tile = a.x + a.y;
-    return fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
+}
+
+// Row maximum of 128 scores (masked ones are -inf).
+__device__ __forceinline__ float row_max(const uint32_t* sr) {
+    float mx8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
+#pragma unroll
+    for (int c = 8; c < 128; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            mx8[i] = fmax3(mx8[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
+    return fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                 fmaxf(mx8[6], mx8[7]));
 }
 
 template <int D>
-__device__ void softmax_epilogue(const AttnParams& p, const Unit& u, Bars* b, uint32_t tmem,
-                                 int X) {
+__device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, int X) {
     using C = Cfg<D>;
-    const AttnStreamDesc& s = p.st[u.si];
     const int wq = (threadIdx.x / 32) & 3;          // TMEM lane quadrant of this warp
     const int r = wq * 32 + (threadIdx.x & 31);     // query row inside the tile
     const uint32_t lane = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane + X * 128;
     const uint32_t tO = tmem + lane + C::kColsO + X * D;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // maximum applied to the exponentials, log2 units
-    float l = 0.f;        // sum of the exponentials (as rounded into P)
-    float l_tile = 0.f;
+    const float ln2 = 0.69314718055994531f;
+    const size_t slot_f = partial_slot_floats(D);
+    int sc = 0;   // S tiles taken, for the s_full phase
+    int oc = 0;   // segments finished, for the o_full phase
+    int ec = 0;   // split epilogues, for the ep_in / ep_out phases
     bool ok = true;
-    for (int j = 0; j < u.n_iter; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->s_full[X]), j & 1, b, p.err));
+    SegIter it(p);
+    Seg g;
+    while (ok && it.next(p, g)) {
+        if (g.rows[X] == 0) continue;  // this segment has no query tile X
+        const AttnStreamDesc& s = p.st[g.si];
+        float m = -INFINITY;  // maximum applied to the exponentials, log2 units
+        float l = 0.f;        // sum of the exponentials (as rounded into P)
+        float l_tile = 0.f;
+        for (int j = 0; j < g.n; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->s_full[X]), sc & 1, b, p.err));
+            if (!ok) break;
+            ++sc;
+            tc_fence_after();
+            uint32_t sr[128];
+            tmem_ld128_wait(tS, sr);
+            const int valid = s.n_k - (g.kt0 + j) * kKeyTile;
+            if (valid < kKeyTile) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+            }
+            if (j == 0) m = row_max(sr) * sl2;  // the running maximum starts here
+            // Exponentials with the maximum in hand (it is not recomputed per
+            // tile).  P and the sums stay finite while no score exceeds m by
+            // 64 or more (log2 units): then p < 2^64 and l < 2^71.  If the
+            // tile's sum leaves that range, the tile is redone against its
+            // exact maximum and O is rescaled, as in the plain online softmax.
+            exp_pass(sr, sl2, m, tS, l_tile);
+            if (__any_sync(0xffffffffu, !(l_tile < 1.8446744e19f))) {
+                const float m_new = fmaxf(m, row_max(sr) * sl2);
+                const float alpha = ex2(m - m_new);
+                l *= alpha;
+                m = m_new;
+                if (j > 0) {
+                    // O holds P V of tiles < j, complete: S(j) was committed after it
+#pragma unroll 1
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t o[32];
+                        tmem_ld32_wait(tO + c, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + c, o);
+                    }
+                }
+                exp_pass(sr, sl2, m, tS, l_tile);
+            }
+            l += l_tile;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->p_full[X]));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->o_full[X]), oc & 1, b, p.err));
+        ++oc;
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld128_wait(tS, sr);
-        const int valid = s.n_k - (u.kt0 + j) * kKeyTile;
-        if (valid < kKeyTile) {
-#pragma unroll
-            for (int c = 0; c < 128; ++c)
-                if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-        }
-        if (j == 0) {
-            // first tile: the running maximum starts from this tile's maximum
-            float mx8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(sr[i]);
-#pragma unroll
-            for (int c = 8; c < 128; c += 16)
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mx8[i] = fmax3(mx8[i], __uint_as_float(sr[c + i]), __uint_as_float(sr[c + 8 + i]));
-            m = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                      fmaxf(mx8[6], mx8[7])) * sl2;
-        }
-        // Exponentials with the maximum in hand; the tile's own maximum is
-        // tracked alongside, off the critical path.  Only if some score rose
-        // more than 8 (log2 units) above m is the tile redone with a larger m.
-        float xmax = exp_pass(sr, sl2, m, tS, l_tile);
-        if (__any_sync(0xffffffffu, xmax > 8.0f)) {
-            const bool need = xmax > 8.0f;
-            const float m_new = need ? m + xmax : m;
-            const float alpha = ex2(m - m_new);
-            l *= alpha;
-            m = m_new;
-            if (j > 0) {
-                // O holds P V of tiles < j, complete: S(j) was committed after it
-#pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t o[32];
-                    tmem_ld32_wait(tO + c, o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + c, o);
-                }
-            }
-            exp_pass(sr, sl2, m, tS, l_tile);
-        }
-        l += l_tile;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->p_full[X]));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->o_full[X]), 0, b, p.err));
-    if (ok) tc_fence_after();
 
-    // ---------------------------------------------------------- epilogue
-    const bool row_ok = ok && r < u.rows[X];
-    const int tok = s.out_tok0 + u.q0 + X * kQRows + r;
-    const float ln2 = 0.69314718055994531f;
-    if (s.n_split == 1) {
+        // ------------------------------------------------------ epilogue
+        const bool row_ok = r < g.rows[X];
+        const int tok = s.out_tok0 + g.q0 + X * kQRows + r;
+        // O leaves TMEM in 32-column chunks: to the output when this CTA
+        // holds the whole item, else to this CTA's partial slot.
+        const bool whole = g.nseg == 1;
         const float inv = 1.0f / l;
-        bf16* dst = p.out + ((size_t)tok * p.heads + u.head) * D;
+        bf16* dst = p.out + ((size_t)tok * p.heads + g.head) * D;
+        float* mine = p.partial + part_slot(p, blockIdx.x, s.cost0 + (long long)(g.head * s.n_qb + g.qb) * s.n_kt, X) * slot_f;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
-            if (ok) {
-                tmem_ld32_wait(tO + c, o);
-            }
-            if (row_ok) {
-                uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+            tmem_ld32_wait(tO + c, o);
+            if (whole) {
+                if (row_ok) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int q = i * 8;
-                    d4[i] = make_uint4(
-                        pack_bf16(__uint_as_float(o[q + 0]) * inv, __uint_as_float(o[q + 1]) * inv),
-                        pack_bf16(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv),
-                        pack_bf16(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv),
-                        pack_bf16(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv));
+                    for (int i = 0; i < 4; ++i) {
+                        const int q = i * 8;
+                        d4[i] = make_uint4(
+                            pack_bf16(__uint_as_float(o[q + 0]) * inv, __uint_as_float(o[q + 1]) * inv),
+                            pack_bf16(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv),
+                            pack_bf16(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv),
+                            pack_bf16(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv));
+                    }
                 }
+            } else {
+                // column-major slot ([D][128], m[128], l[128]): a warp stores 32
+                // consecutive floats
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    __stcg(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]));
             }
         }
-        if (row_ok && p.lse) p.lse[(size_t)tok * p.heads + u.head] = (m + __log2f(l)) * ln2;
-        return;
-    }
-
-    // split-KV: store the unnormalised partial, the last of the parts merges.
-    // A slot is column-major ([D][128] then m[128], l[128]) so that the 32
-    // lanes of a warp always touch 32 consecutive floats.
-    const size_t slot_f = partial_slot_floats(D);
-    const int tile_id = (u.head * s.n_qb + u.qb) * kQTilesPerCta + X;
-    const size_t slot0 = (size_t)s.part0 + (size_t)tile_id * s.n_split;
-    float* mine = p.partial + (slot0 + u.split) * slot_f;
-#pragma unroll 1
-    for (int c = 0; c < D; c += 32) {
-        uint32_t o[32];
-        if (ok) tmem_ld32_wait(tO + c, o);
-        if (ok) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) __stcg(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]));
+        // O is read out: the next segment's first P V may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->o_empty[X]));
+        if (whole) {
+            if (row_ok && p.lse) p.lse[(size_t)tok * p.heads + g.head] = (m + __log2f(l)) * ln2;
+            continue;
         }
-    }
-    if (ok) {
         __stcg(mine + (size_t)kQRows * D + r, m);
         __stcg(mine + (size_t)kQRows * D + kQRows + r, l);
-    }
-    __threadfence();
-    named_sync(1 + X, 128);
-    if (r == 0) {
-        int last = 0;
-        if (ok && !*(volatile int*)&b->abort) {
-            int* cnt = p.counters + s.cnt0 + tile_id;
-            const int old = atomicAdd(cnt, 1);
-            last = old == s.n_split - 1;
-            if (last) *cnt = 0;  // ready for the next launch
+        // all four warps' partial rows are visible before the arrival count
+        // moves; bounded waits on mbarriers, not bar.sync, so that an
+        // aborting CTA can never block here
+        __threadfence();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->ep_in[X]));
+        if (r == 0) {
+            int last = 0;
+            if (mbar_wait(smem_u32(&b->ep_in[X]), ec & 1, b, p.err) &&
+                !*(volatile int*)&b->abort) {
+                int* cnt = p.counters + (size_t)g.item * kQTilesPerCta + X;
+                const int old = atomicAdd(cnt, 1);
+                last = old == g.nseg - 1;
+                if (last) *cnt = 0;  // ready for the next launch
+            }
+            b->last[X] = last;
+            mbar_arrive(smem_u32(&b->ep_out[X]));
         }
-        b->last[X] = last;
-    }
-    named_sync(1 + X, 128);
-    if (!b->last[X] || !row_ok) return;
-    __threadfence();
-    float M = -INFINITY;
-    for (int i = 0; i < s.n_split; ++i)
-        M = fmaxf(M, __ldcg(p.partial + (slot0 + i) * slot_f + (size_t)kQRows * D + r));
-    float L = 0.f;
-    for (int i = 0; i < s.n_split; ++i) {
-        const float* pi = p.partial + (slot0 + i) * slot_f;
-        L += __ldcg(pi + (size_t)kQRows * D + kQRows + r) * ex2(__ldcg(pi + (size_t)kQRows * D + r) - M);
-    }
-    const float invL = 1.0f / L;
-    bf16* dst = p.out + ((size_t)tok * p.heads + u.head) * D;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->ep_out[X]), ec & 1, b, p.err));
+        ++ec;
+        if (!ok) break;
+        if (!b->last[X] || !row_ok) continue;
+        __threadfence();
+        // the parts of this item: CTAs c_first .. c_first + nseg - 1
+        const long long i0 = s.cost0 + (long long)(g.head * s.n_qb + g.qb) * s.n_kt;
+        float M = -INFINITY;
+        for (int k = 0; k < g.nseg; ++k) {
+            const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
+            M = fmaxf(M, __ldcg(pk + (size_t)kQRows * D + r));
+        }
+        float L = 0.f;
+        for (int k = 0; k < g.nseg; ++k) {
+            const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
+            L += __ldcg(pk + (size_t)kQRows * D + kQRows + r) * ex2(__ldcg(pk + (size_t)kQRows * D + r) - M);
+        }
+        const float invL = 1.0f / L;
 #pragma unroll 1
-    for (int c = 0; c < D; c += 16) {
-        float acc[16];
+        for (int c = 0; c < D; c += 16) {
+            float acc[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-        for (int i = 0; i < s.n_split; ++i) {
-            const float* pi = p.partial + (slot0 + i) * slot_f;
-            const float w = ex2(__ldcg(pi + (size_t)kQRows * D + r) - M) * invL;
-            float v[16];
+            for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+            for (int k = 0; k < g.nseg; ++k) {
+                const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
+                const float w = ex2(__ldcg(pk + (size_t)kQRows * D + r) - M) * invL;
+                float v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __ldcg(pi + (size_t)(c + k) * kQRows + r);
+                for (int q = 0; q < 16; ++q) v[q] = __ldcg(pk + (size_t)(c + q) * kQRows + r);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k] = fmaf(w, v[k], acc[k]);
+                for (int q = 0; q < 16; ++q) acc[q] = fmaf(w, v[q], acc[q]);
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+            d4[0] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                               pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+            d4[1] = make_uint4(pack_bf16(acc[8], acc[9]), pack_bf16(acc[10], acc[11]),
+                               pack_bf16(acc[12], acc[13]), pack_bf16(acc[14], acc[15]));
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-        d4[0] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
-                           pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
-        d4[1] = make_uint4(pack_bf16(acc[8], acc[9]), pack_bf16(acc[10], acc[11]),
-                           pack_bf16(acc[12], acc[13]), pack_bf16(acc[14], acc[15]));
+        if (p.lse) p.lse[(size_t)tok * p.heads + g.head] = (M + __log2f(L)) * ln2;
     }
-    if (p.lse) p.lse[(size_t)tok * p.heads + u.head] = (M + __log2f(L)) * ln2;
 }
 
 template <int D>
@@ -638,16 +717,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Bars* b = reinterpret_cast<Bars*>(smem + C::kBarOff);
-    const Unit u = decode_unit(p);
-    if (u.si < 0) return;  // the same for every thread of the CTA
     const int warp = threadIdx.x / 32;
     const int lane_id = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&b->q_full), 1);
+        mbar_init(smem_u32(&b->q_empty), 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&b->s_full[x]), 1);
-            mbar_init(smem_u32(&b->p_full[x]), 4);  // one arrive per softmax warp
+            mbar_init(smem_u32(&b->p_full[x]), 4);   // one arrive per softmax warp
             mbar_init(smem_u32(&b->o_full[x]), 1);
+            mbar_init(smem_u32(&b->o_empty[x]), 4);  // one arrive per softmax warp
+            mbar_init(smem_u32(&b->ep_in[x]), 4);
+            mbar_init(smem_u32(&b->ep_out[x]), 1);
         }
         mbar_init(smem_u32(&b->mma_done), 1);
         for (int i = 0; i < C::kStages; ++i) {
@@ -673,15 +754,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
         if (warp == 0) {
-            if (lane_id == 0) producer<D>(&tq, &tk, &tv, p, u, smem, b);
+            if (lane_id == 0) producer<D>(&tq, &tk, &tv, p, smem, b);
         } else if (warp == 1) {
-            if (lane_id == 0) mma_issuer<D>(p, u, smem, b, tmem);
+            if (lane_id == 0) mma_issuer<D>(p, smem, b, tmem);
             __syncwarp();
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-        const int X = warp / 4 - 1;
-        if (X == 0 || u.rows[1] > 0) softmax_epilogue<D>(p, u, b, tmem, X);
+        softmax_epilogue<D>(p, b, tmem, warp / 4 - 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -694,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const AttnParams& p, int n_units, cudaStream_t s) {
+                     const AttnParams& p, cudaStream_t s) {
     using C = Cfg<D>;
     static bool configured = false;
     if (!configured) {
@@ -703,17 +783,17 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    attn_kernel<D><<<n_units, kThreads, C::kSmem, s>>>(tq, tk, tv, p);
+    attn_kernel<D><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, int n_units, cudaStream_t s) {
-    if (n_units <= 0) return cudaErrorInvalidValue;
-    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, p, n_units, s);
-    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, p, n_units, s);
+                        const AttnParams& p, cudaStream_t s) {
+    if (p.grid <= 0 || p.total <= 0) return cudaErrorInvalidValue;
+    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, p, s);
+    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, p, s);
     return cudaErrorInvalidValue;
 }
 

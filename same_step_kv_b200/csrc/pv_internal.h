@@ -20,7 +20,7 @@ constexpr int kQRows = 128;               // query rows per tensor-core tile (MM
 constexpr int kQTilesPerCta = 2;          // two query tiles share each K/V tile
 constexpr int kQBlock = kQRows * kQTilesPerCta;
 constexpr int kKeyTile = 128;             // keys per K/V tile (MMA N of Q K^T)
-constexpr int kMaxSplit = 32;             // split-KV parts of one query tile
+constexpr int kMaxGrid = 160;             // CTAs of one attention launch at most (>= SMs)
 
 // ---------------------------------------------------------------- RoPE + append
 struct RopeStreamDesc {
@@ -60,22 +60,27 @@ struct AttnStreamDesc {
     int out_tok0;        // first token row of out / lse
     int n_qb;            // query blocks of kQBlock rows
     int n_kt;            // key tiles
-    int n_split;         // key-range parts per query block
-    int unit0;           // first CTA index of this stream
-    int part0;           // first partial-result slot
-    int cnt0;            // first arrival counter
+    int item0;           // global index of this stream's first (head, query block) item
+    long long cost0;     // key tiles of all items before this stream's first
 };
 
+// One launch is a stream-K schedule: the items (head, query block) of all
+// streams, in order, each costing n_kt key tiles, laid end to end; CTA c
+// of `grid` processes the key tiles [c*total/grid, (c+1)*total/grid).
 struct AttnParams {
     bf16* out;
     float* lse;
-    float* partial;      // split-KV partial results (unnormalised O, m, l)
-    int* counters;       // arrivals per query tile; the last arriver resets to 0
+    float* partial;      // split-KV partial results, 4 slots per CTA (unnormalised O, m, l)
+    int* counters;       // arrivals per (item, query tile); the last arriver resets to 0
     int* err;            // device error word (bounded waits that gave up)
     int heads;
     int head_dim;
     float scale_log2;    // log2(e) / sqrt(D)
     int n_streams;
+    int grid;            // CTAs of the launch
+    int item_aligned;    // 1: CTA ranges end on item boundaries (no partial results)
+    int n_items;         // items of all streams
+    long long total;     // key tiles of all items
     AttnStreamDesc st[PV_MAX_STREAMS];
 };
 
@@ -83,7 +88,7 @@ struct AttnParams {
 __host__ __device__ inline size_t partial_slot_floats(int D) { return (size_t)kQRows * D + 2 * kQRows; }
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, int n_units, cudaStream_t s);
+                        const AttnParams& p, cudaStream_t s);
 
 // ----------------------------------------------------------------- Euler
 cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaStream_t s);
@@ -97,9 +102,11 @@ bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, 
 // Records a failure for pv_last_error() and returns code.
 pv_status report_error(pv_status code, const char* msg);
 
-// Split-KV plan for one attention launch: fills n_split, unit0, part0, cnt0.
-// Returns the number of CTAs, or -1 when the partial slots do not suffice.
-int plan_attention(AttnStreamDesc* st, int n_streams, int heads, int n_sm, int part_capacity,
-                   int cnt_capacity, int* order);
+// Stream-K plan for one attention launch: fills n_qb, n_kt, item0, cost0 of
+// every stream and grid, total, n_items, item_aligned of p.  Returns the
+// number of CTAs, or -1 when the counters (2 per item) do not fit.  When the
+// partial slots (4 per CTA) do not suffice for one CTA per SM, the CTAs take
+// whole items instead (item_aligned) and need none.
+int plan_attention(AttnParams& p, int n_sm, int part_capacity, int cnt_capacity);
 
 }  // namespace pv

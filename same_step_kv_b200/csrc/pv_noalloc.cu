@@ -13,8 +13,8 @@
 // The scratch is one file-scope device array of kScratchBytes (8 MiB) that
 // every GPU loading this library holds until the process exits.  It holds an
 // error word, the split-KV arrival counters (at most kMaxCounters query
-// tiles) and as many partial-result slots as fit; the planner splits the key
-// range only as far as those slots allow.
+// tiles) and as many partial-result slots as fit; when they do not suffice for
+// one CTA per SM, the planner gives each CTA whole query blocks instead.
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -134,16 +134,14 @@ extern "C" pv_status pv_attn_dense_noalloc(const void* q, const void* k, const v
     a.kv_row0 = 0;
     a.kv_head_stride = n_k;
     a.out_tok0 = 0;
-    int order[1];
-    const int units = plan_attention(p.st, 1, heads, n_sm, n_part, kMaxCounters, order);
-    if (units < 0)
+    if (plan_attention(p, n_sm, n_part, kMaxCounters) < 0)
         return report_error(PV_ERR_CAPACITY, "pv_attn_dense_noalloc: no plan fits the scratch");
     CUtensorMap tq, tk, tv;
     if (!encode_rows_map(&tq, q, (long long)heads * n_q, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tk, k, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg))
         return report_error(PV_ERR_CUDA, msg);
-    e = launch_attn(tq, tk, tv, p, units, st);
+    e = launch_attn(tq, tk, tv, p, st);
     if (e != cudaSuccess) {
         snprintf(msg, sizeof msg, "pv_attn_dense_noalloc launch: %s", cudaGetErrorString(e));
         return report_error(PV_ERR_CUDA, msg);
