@@ -63,7 +63,7 @@ struct Bars {  // 264 bytes, inside the 512 reserved after the tiles
     uint64_t o_full[2];
     uint64_t mma_done;
     uint64_t kv_full[8];
-    uint64_t kv_empty[8];
+    uint64_t rel[8];      // release events: the K/V tiles they free may be overwritten
     uint32_t tmem_base;
     int abort;
     int last[2];
@@ -341,6 +341,8 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     using C = Cfg<D>;
     const uint32_t qbar = smem_u32(&b->q_full);
     int kv = 0, qseg = 0;
+    int ev0 = 0;              // first release event of the current segment
+    int stage_ev[C::kStages]; // release event of the tile in each stage
     bool ok = true;
     SegIter it(p);
     Seg g;
@@ -360,8 +362,14 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
         for (int j = 0; ok && j < g.n; ++j) {
             for (int w = 0; w < 2; ++w) {
                 const int st = kv % C::kStages;
-                const uint32_t ph = (kv / C::kStages) & 1;
-                if (!(ok = mbar_wait(smem_u32(&b->kv_empty[st]), ph ^ 1, b, p.err))) break;
+                // the tile loaded kStages loads ago must have been released
+                if (kv >= C::kStages) {
+                    const int e = stage_ev[st];
+                    if (!(ok = mbar_wait(smem_u32(&b->rel[e & 7]), (e >> 3) & 1, b, p.err))) break;
+                }
+                // K_j is released at the end of iteration j, V_j at the end of
+                // iteration j + 1 (or of the segment)
+                stage_ev[st] = ev0 + j + w;
                 const uint32_t full = smem_u32(&b->kv_full[st]);
                 mbar_expect_tx(full, C::kTileBytes);
                 const CUtensorMap* m = w == 0 ? tk : tv;
@@ -371,6 +379,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
                 ++kv;
             }
         }
+        ev0 += g.n + 1;
     }
     // Before leaving, make sure no copy of ours is still landing in shared
     // memory: wait (bounded) for the last load issued into each stage, and
@@ -416,6 +425,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
                    (acc || kk > 0) ? 1u : 0u);
     };
     int kv = 0, qseg = 0;
+    int ev0 = 0;         // first release event of the current segment
     int pc[2] = {0, 0};  // P tiles consumed, per query tile
     int oc[2] = {0, 0};  // segments finished, per query tile
     bool ok = true;
@@ -457,8 +467,8 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
                 qk(1, ks);
                 tc_commit(smem_u32(&b->s_full[1]));
             }
-            if (j > 0) tc_commit(smem_u32(&b->kv_empty[vs_prev]));
-            tc_commit(smem_u32(&b->kv_empty[ks]));
+            // one release per iteration: K_j and V_(j-1) are no longer read
+            tc_commit(smem_u32(&b->rel[(ev0 + j) & 7]));
         }
         if (!ok) break;
         tc_commit(smem_u32(&b->q_empty));  // the Q tiles are free once these S products end
@@ -473,8 +483,9 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
             tc_commit(smem_u32(&b->o_full[1]));
             ++oc[1];
         }
-        tc_commit(smem_u32(&b->kv_empty[vs]));
+        tc_commit(smem_u32(&b->rel[(ev0 + n) & 7]));  // V of the last iteration
         kv += 2 * n;
+        ev0 += n + 1;
     }
     // every MMA issued by this thread has completed once mma_done flips
     tc_commit(smem_u32(&b->mma_done));
@@ -731,10 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&b->ep_out[x]), 1);
         }
         mbar_init(smem_u32(&b->mma_done), 1);
-        for (int i = 0; i < C::kStages; ++i) {
-            mbar_init(smem_u32(&b->kv_full[i]), 1);
-            mbar_init(smem_u32(&b->kv_empty[i]), 1);
-        }
+        for (int i = 0; i < C::kStages; ++i) mbar_init(smem_u32(&b->kv_full[i]), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(smem_u32(&b->rel[i]), 1);
         b->abort = 0;
         b->last[0] = b->last[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
