@@ -311,3 +311,42 @@ def test_euler_straight_line_lands_on_data():
         x = euler.euler_step(x, v, sig[i], sig[i + 1])
         np.testing.assert_allclose(x, (1 - sig[i + 1]) * x0 + sig[i + 1] * x1, atol=1e-14)
     np.testing.assert_allclose(x, x0, atol=1e-14)
+
+
+# --------------------------------------------------------- sampler variants
+
+
+def test_shift_schedule_reproduces_printed_timesteps():
+    g = load("shift_schedule.txt")
+    sig = euler.shifted_schedule(g["steps"], g["shift"])
+    t = euler.timesteps(sig[:-1])
+    assert list(t[:6]) == [g[f"t{i}"] for i in range(6)]
+    assert int((t >= g["high_noise_boundary"]).sum()) == g["steps_at_or_above_boundary"]
+    assert int((t < g["high_noise_boundary"]).sum()) == g["steps_below_boundary"]
+    # "half of the sampling points fall in the t > 926 interval"
+    assert int((1000 * sig[:-1] > g["median_boundary"]).sum()) == g["steps"] // 2
+    assert sig[-1] == 0.0 and np.all(np.diff(sig) < 0)
+
+
+def test_shift_transform_properties():
+    # identity at shift 1, fixed ends 0 and 1, and shift > 1 pushes every interior
+    # point toward the noise end (chapter 5)
+    s = np.linspace(0.0, 1.0, 101)
+    np.testing.assert_allclose(euler.shift_sigma(s, 1.0), s, atol=0)
+    for k in (3.0, 5.0, 12.0):
+        y = euler.shift_sigma(s, k)
+        assert y[0] == 0.0 and y[-1] == 1.0
+        assert np.all(y[1:-1] > s[1:-1])
+        # the inverse map is the same transform with 1/shift
+        np.testing.assert_allclose(euler.shift_sigma(y, 1.0 / k), s, atol=1e-15)
+
+
+def test_cfg_combine_special_cases():
+    u = synth.normal_f32(41, (1000,)).double().numpy()
+    c = synth.normal_f32(42, (1000,)).double().numpy()
+    np.testing.assert_array_equal(euler.cfg_combine(u, c, 0.0), u)          # w = 0: unconditional
+    np.testing.assert_allclose(euler.cfg_combine(u, c, 1.0), c, atol=1e-15)  # w = 1: conditional
+    np.testing.assert_allclose(euler.cfg_combine(u, u, 7.5), u, atol=0)      # no difference
+    # linear in w
+    a, b = euler.cfg_combine(u, c, 2.0), euler.cfg_combine(u, c, 4.0)
+    np.testing.assert_allclose(b - a, 2.0 * (c - u), atol=1e-13)
