@@ -200,6 +200,7 @@ def main():
     import torch
     import torch.distributed as dist
     from same_step_kv_b200 import pv, synth
+    from same_step_kv_b200.dist import max_over_ranks
 
     torch.cuda.set_device(local)
     if world > 1:
@@ -260,12 +261,7 @@ def main():
         torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-        if rank == 0:
-            pass
+    ms = max_over_ranks(ms)       # the slowest rank sets the job's time
     ms_step = ms / args.steps
 
     # ---- e2e: the same step through the public API from pinned host buffers
@@ -309,10 +305,7 @@ def main():
     e1.record(cs)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms)
     h2d = NL * 3 * T * HEADS * D * 2 + LATENT * 4
     d2h = LATENT * 4
 

@@ -209,6 +209,32 @@ PV_API pv_status pv_attn_dense(const void* q, const void* k, const void* v, int 
                         int heads, int head_dim, void* out, float* lse, void* ws,
                         size_t ws_bytes, void* cuda_stream);
 
+/* Workspace bytes that pv_attn_varlen needs for these sequence lengths. */
+PV_API pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* n_k, int heads,
+                                         int head_dim, size_t* ws_bytes);
+
+/* Softmax attention of n_seqs independent sequences of ragged lengths in one
+ * launch, the same kernel as pv_attn_dense.  Its use here is the DiT's
+ * cross-attention (blog chapter 3, "Where Did the Prompt Go?": each layer's
+ * video tokens query the prompt's text context, up to 512 vectors, trimmed
+ * to the prompt's real length; chapter 4: the context holds no sequence
+ * positions, so no RoPE, and no mask), one sequence per prompt.
+ *  n_q, n_k: HOST arrays of n_seqs lengths (1 <= n_seqs <= PV_MAX_STREAMS);
+ *    n_q[i] = 0 skips sequence i; n_q[i] > 0 needs n_k[i] >= 1.
+ *  q: the sequences' head-major blocks back to back, bf16: block i is
+ *    [H][n_q[i]][D] and starts at row H * (n_q[0] + ... + n_q[i-1]).
+ *  k, v: likewise [H][n_k[i]][D] blocks.  Rows past a block's last key inside
+ *    a 128-key tile are read from the next block (or as zeros past the
+ *    buffer) and masked out, so k and v must hold finite values.
+ *  out: bf16 [sum n_q][H][D], token-major, sequence i from token
+ *    n_q[0] + ... + n_q[i-1].  lse: optional f32 [sum n_q][H].
+ *  ws: device workspace of pv_attn_varlen_ws_bytes bytes, zero-filled before
+ *    its first use, 256-byte aligned. */
+PV_API pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs,
+                                const int* n_q, const int* n_k, int heads, int head_dim,
+                                void* out, float* lse, void* ws, size_t ws_bytes,
+                                void* cuda_stream);
+
 /* Dense attention like pv_attn_dense (same layouts, same kernel), for
  * callers that cannot allocate device memory where they call it: code inside
  * a custom allocator or memory-pool callback, plugins whose host framework
@@ -235,6 +261,29 @@ PV_API pv_status pv_attn_dense_noalloc(const void* q, const void* k, const void*
  *  caller in fp64 and passed rounded to f32. */
 PV_API pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* cuda_stream);
 
+/* Shifted sigma schedule of n_steps denoising steps (blog chapter 5, "shift:
+ * Where the 40 Stops Land"): a uniform grid u_i = sigma_max * (1 - i/n_steps),
+ * i < n_steps, mapped by sigma = shift * u / (1 + (shift - 1) * u), then a
+ * final 0.  sigmas_out: host array of n_steps + 1 doubles.  timesteps_out
+ * (optional, n_steps ints): floor(1000 * sigma_i), the 1000-tick scale of
+ * the blog's chapter 1.  sigma_max <= 0 selects 1 - 1/1000, which with shift
+ * 12 and 40 steps gives the blog's printed 999, 997, 995, 993, 990, 988.
+ * Host only, fp64. */
+PV_API pv_status pv_sigma_schedule(int n_steps, double shift, double sigma_max,
+                                   double* sigmas_out, int* timesteps_out);
+
+/* Euler update on the classifier-free-guided velocity, in place (blog
+ * chapter 5, "CFG"): x[i] += dsigma * (v_uncond[i] + guide_scale *
+ * (v_cond[i] - v_uncond[i])), f32; the guided velocity is never stored. */
+PV_API pv_status pv_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond,
+                                   size_t n, float guide_scale, float dsigma,
+                                   void* cuda_stream);
+
+/* Clean-data estimate of flow matching (blog chapter 1): x0[i] = x[i] -
+ * sigma * v[i], f32, one fused multiply-add per element; x0 may alias x. */
+PV_API pv_status pv_x0_estimate(float* x0, const float* x, const float* v, size_t n,
+                                float sigma, void* cuda_stream);
+
 /* Self-test of the attention kernel's software exponential: y[i] = 2^x[i]
  * computed as that kernel computes a quarter of its softmax exponentials
  * (round-to-nearest range reduction and a fitted minimax cubic; maximum
@@ -244,8 +293,17 @@ PV_API pv_status pv_selftest_exp2_poly(const float* x, float* y, size_t n, void*
 
 /* Reads (synchronously) and clears the device error word that the kernels of
  * this handle set when a bounded device-side wait gives up.  *code is 0 when
- * no wait timed out. */
+ * no wait timed out; otherwise the call returns PV_ERR_TIMEOUT and also
+ * re-zeroes the workspace's split-merge arrival counters, which an aborted
+ * launch may have left part counted. */
 PV_API pv_status pv_kv_poll_device_error(pv_kv kv, int* code);
+
+/* Failure-path self-test: launches one device-side wait on a barrier that
+ * nothing ever arrives on.  Like every wait of the attention kernel it gives
+ * up after about one second, records a timeout in this handle's device error
+ * word and returns, leaving the GPU context usable; pv_kv_poll_device_error
+ * then reports PV_ERR_TIMEOUT.  Asynchronous on cuda_stream. */
+PV_API pv_status pv_kv_selftest_wait_timeout(pv_kv kv, void* cuda_stream);
 
 #ifdef __cplusplus
 }

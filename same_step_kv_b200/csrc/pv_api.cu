@@ -255,6 +255,30 @@ pv_status q_map(pv_kv kv, const void* q_rot, long long rows, CUtensorMap* out) {
     return PV_OK;
 }
 
+// Shape checks and sizes shared by pv_attn_varlen_ws_bytes and pv_attn_varlen.
+pv_status varlen_sizes(int n_seqs, const int* n_q, const int* n_k, int heads, int head_dim,
+                       long long* tot_q, long long* tot_k, size_t* n_cnt, size_t* tiles) {
+    if (!n_q || !n_k) return fail(PV_ERR_INVALID_ARG, "NULL length array");
+    if (n_seqs < 1 || n_seqs > PV_MAX_STREAMS)
+        return fail(PV_ERR_SHAPE, "n_seqs %d outside 1..%d", n_seqs, PV_MAX_STREAMS);
+    if (heads < 1 || (head_dim != 64 && head_dim != 128))
+        return fail(PV_ERR_SHAPE, "heads must be positive and head_dim 64 or 128");
+    *tot_q = *tot_k = 0;
+    *n_cnt = *tiles = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        if (n_q[i] < 0 || n_k[i] < 0 || (n_q[i] > 0 && n_k[i] == 0))
+            return fail(PV_ERR_SHAPE, "sequence %d: n_q %d, n_k %d (queries need keys)", i, n_q[i],
+                        n_k[i]);
+        const size_t qb = (n_q[i] + kQBlock - 1) / kQBlock;
+        *n_cnt += (size_t)heads * qb * kQTilesPerCta;
+        *tiles += (size_t)heads * qb * ((n_k[i] + kKeyTile - 1) / kKeyTile);
+        *tot_q += n_q[i];
+        *tot_k += n_k[i];
+    }
+    if (*tot_q * heads >= (1LL << 31) || *tot_k * heads >= (1LL << 31))
+        return fail(PV_ERR_SHAPE, "too many rows for a tensor map");
+    return PV_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -706,6 +730,79 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
     return PV_OK;
 }
 
+pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* n_k, int heads,
+                                  int head_dim, size_t* ws_bytes) {
+    if (!ws_bytes) return fail(PV_ERR_INVALID_ARG, "output pointer is NULL");
+    long long tq, tk;
+    size_t n_cnt, tiles;
+    pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, head_dim, &tq, &tk, &n_cnt, &tiles);
+    if (st) return st;
+    const size_t n_part = 4 * std::min<size_t>(kMaxGrid, std::max<size_t>(tiles, 1));
+    *ws_bytes = 256 + round_up(std::max<size_t>(n_cnt, 1) * sizeof(int), 256) +
+                n_part * partial_slot_floats(head_dim) * sizeof(float);
+    return PV_OK;
+}
+
+pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs, const int* n_q,
+                         const int* n_k, int heads, int head_dim, void* out, float* lse, void* ws,
+                         size_t ws_bytes, void* cuda_stream) {
+    long long tot_q, tot_k;
+    size_t n_cnt, tiles;
+    pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, head_dim, &tot_q, &tot_k, &n_cnt, &tiles);
+    if (st) return st;
+    if (tot_q == 0) return PV_OK;  // no queries: nothing to compute
+    if (!q || !k || !v || !out) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return fail(PV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    size_t need = 0;
+    pv_attn_varlen_ws_bytes(n_seqs, n_q, n_k, heads, head_dim, &need);
+    if (!ws || ws_bytes < need || !aligned(ws, 256))
+        return fail(PV_ERR_CAPACITY, "workspace of %zu bytes at %p, need %zu (256-byte aligned)",
+                    ws_bytes, ws, need);
+    if ((st = check_async("an earlier launch"))) return st;
+    int n_sm = 148;
+    if ((st = check_device(&n_sm))) return st;
+    const int n_part = (int)(4 * std::min<size_t>(kMaxGrid, tiles));
+    AttnParams p{};
+    p.out = (bf16*)out;
+    p.lse = lse;
+    p.err = (int*)ws;
+    p.counters = (int*)((char*)ws + 256);
+    p.partial = (float*)((char*)ws + 256 + round_up(n_cnt * sizeof(int), 256));
+    p.heads = heads;
+    p.head_dim = head_dim;
+    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
+    // sequence i: queries at head-major rows heads*qoff + h*n_q[i], keys at
+    // heads*koff + h*n_k[i]; sequences without queries get no descriptor
+    int ns = 0;
+    long long qoff = 0, koff = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        if (n_q[i] > 0) {
+            AttnStreamDesc& a = p.st[ns++];
+            a.n_q = n_q[i];
+            a.n_k = n_k[i];
+            a.q_row0 = (int)(heads * qoff);
+            a.kv_row0 = (int)(heads * koff);
+            a.kv_head_stride = n_k[i];
+            a.out_tok0 = (int)qoff;
+        }
+        qoff += n_q[i];
+        koff += n_k[i];
+    }
+    p.n_streams = ns;
+    if (plan_attention(p, n_sm, n_part, (int)n_cnt) < 0)
+        return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
+    CUtensorMap tq, tk, tv;
+    char msg[256];
+    if (!encode_rows_map(&tq, q, heads * tot_q, head_dim, msg, sizeof msg) ||
+        !encode_rows_map(&tk, k, heads * tot_k, head_dim, msg, sizeof msg) ||
+        !encode_rows_map(&tv, v, heads * tot_k, head_dim, msg, sizeof msg))
+        return fail(PV_ERR_CUDA, "%s", msg);
+    cudaError_t e = launch_attn(tq, tk, tv, p, (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attn_varlen launch");
+    return PV_OK;
+}
+
 pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* cuda_stream) {
     if (n == 0) return PV_OK;
     if (!x || !v) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -718,6 +815,51 @@ pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* 
     return PV_OK;
 }
 
+pv_status pv_sigma_schedule(int n_steps, double shift, double sigma_max, double* sigmas_out,
+                            int* timesteps_out) {
+    if (n_steps < 1 || !sigmas_out) return fail(PV_ERR_INVALID_ARG, "n_steps < 1 or NULL output");
+    if (!(shift > 0.0) || !std::isfinite(shift)) return fail(PV_ERR_INVALID_ARG, "shift must be > 0");
+    if (sigma_max <= 0.0) sigma_max = 1.0 - 1.0 / 1000.0;
+    if (!(sigma_max <= 1.0)) return fail(PV_ERR_INVALID_ARG, "sigma_max must be in (0, 1]");
+    for (int i = 0; i < n_steps; ++i) {
+        const double u = sigma_max * (1.0 - (double)i / n_steps);
+        sigmas_out[i] = shift * u / (1.0 + (shift - 1.0) * u);
+        if (timesteps_out) timesteps_out[i] = (int)std::floor(1000.0 * sigmas_out[i]);
+    }
+    sigmas_out[n_steps] = 0.0;
+    return PV_OK;
+}
+
+pv_status pv_euler_cfg_step(float* x, const float* v_cond, const float* v_uncond, size_t n,
+                            float guide_scale, float dsigma, void* cuda_stream) {
+    if (n == 0) return PV_OK;
+    if (!x || !v_cond || !v_uncond) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned(x, 4) || !aligned(v_cond, 4) || !aligned(v_uncond, 4))
+        return fail(PV_ERR_INVALID_ARG, "misaligned f32 tensor");
+    if (!std::isfinite(dsigma) || !std::isfinite(guide_scale))
+        return fail(PV_ERR_INVALID_ARG, "dsigma and guide_scale must be finite");
+    pv_status st;
+    if ((st = check_async("an earlier launch"))) return st;
+    cudaError_t e = launch_euler_cfg(x, v_cond, v_uncond, n, guide_scale, dsigma,
+                                     (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "euler_cfg launch");
+    return PV_OK;
+}
+
+pv_status pv_x0_estimate(float* x0, const float* x, const float* v, size_t n, float sigma,
+                         void* cuda_stream) {
+    if (n == 0) return PV_OK;
+    if (!x0 || !x || !v) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned(x0, 4) || !aligned(x, 4) || !aligned(v, 4))
+        return fail(PV_ERR_INVALID_ARG, "misaligned f32 tensor");
+    if (!std::isfinite(sigma)) return fail(PV_ERR_INVALID_ARG, "sigma must be finite");
+    pv_status st;
+    if ((st = check_async("an earlier launch"))) return st;
+    cudaError_t e = launch_x0(x0, x, v, n, sigma, (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "x0 launch");
+    return PV_OK;
+}
+
 pv_status pv_kv_poll_device_error(pv_kv kv, int* code) {
     if (!kv || !code) return fail(PV_ERR_INVALID_ARG, "NULL argument");
     *code = 0;
@@ -725,11 +867,25 @@ pv_status pv_kv_poll_device_error(pv_kv kv, int* code) {
     cudaError_t e = cudaMemcpy(code, kv->ws + kv->wl.err_off, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
     if (*code) {
-        const int zero = 0;
-        e = cudaMemcpy(kv->ws + kv->wl.err_off, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        // an aborted launch may leave split-merge arrival counters part
+        // counted: clear them with the error word
+        e = cudaMemset(kv->ws + kv->wl.err_off, 0, sizeof(int));
+        if (e == cudaSuccess)
+            e = cudaMemset(kv->ws + kv->wl.cnt_off, 0, sizeof(int) * (size_t)kv->wl.n_counters);
         if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
         return fail(PV_ERR_TIMEOUT, "a device-side wait gave up (code %d)", *code);
     }
+    return PV_OK;
+}
+
+pv_status pv_kv_selftest_wait_timeout(pv_kv kv, void* cuda_stream) {
+    if (!kv) return fail(PV_ERR_INVALID_ARG, "handle is NULL");
+    if (!kv->device) return fail(PV_ERR_STATE, "bookkeeping-only handle has no device buffers");
+    pv_status st;
+    if ((st = check_async("an earlier launch"))) return st;
+    cudaError_t e = launch_wait_timeout_probe((int*)(kv->ws + kv->wl.err_off),
+                                              (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait-timeout self-test launch");
     return PV_OK;
 }
 

@@ -288,6 +288,7 @@ __device__ __forceinline__ int cta_of(const AttnParams& p, long long x) {
 struct Seg {
     int si, head, qb, kt0, n, q0, rows[2];
     int item;      // global item index
+    long long i0;  // the item's first key tile in the launch's tile sequence
     int c_first;   // first CTA holding part of the item
     int nseg;      // CTAs holding parts of the item
     int which;     // 0: this CTA's first segment, 1: a later one
@@ -310,9 +311,13 @@ struct SegIter {
         const long long e = i1 < end ? i1 : end;
         g.n = (int)(e - pos);
         g.which = pos == bound(p, blockIdx.x) ? 0 : 1;
-        g.head = li / s.n_qb;
-        g.qb = li - g.head * s.n_qb;
+        // items are laid out query-block-major: with a grid that is a multiple
+        // of n_qb, the CTAs working on one head's query blocks then walk the
+        // same key tiles at the same time and share them through L2
+        g.qb = li / p.heads;
+        g.head = li - g.qb * p.heads;
         g.item = s.item0 + li;
+        g.i0 = i0;
         if (p.item_aligned) {
             g.c_first = blockIdx.x;
             g.nseg = 1;
@@ -623,7 +628,7 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         const bool whole = g.nseg == 1;
         const float inv = 1.0f / l;
         bf16* dst = p.out + ((size_t)tok * p.heads + g.head) * D;
-        float* mine = p.partial + part_slot(p, blockIdx.x, s.cost0 + (long long)(g.head * s.n_qb + g.qb) * s.n_kt, X) * slot_f;
+        float* mine = p.partial + part_slot(p, blockIdx.x, g.i0, X) * slot_f;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
@@ -683,7 +688,7 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         if (!b->last[X] || !row_ok) continue;
         __threadfence();
         // the parts of this item: CTAs c_first .. c_first + nseg - 1
-        const long long i0 = s.cost0 + (long long)(g.head * s.n_qb + g.qb) * s.n_kt;
+        const long long i0 = g.i0;
         float M = -INFINITY;
         for (int k = 0; k < g.nseg; ++k) {
             const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
@@ -796,7 +801,25 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     return cudaGetLastError();
 }
 
+// One bounded wait on an mbarrier that nothing arrives on: it gives up after
+// kWaitCycles, records the timeout in *err and returns, exactly as a wait of
+// attn_kernel does; used to check the failure path without a GPU fault.
+__global__ void wait_timeout_kernel(int* err) {
+    __shared__ Bars b;
+    if (threadIdx.x == 0) {
+        b.abort = 0;
+        mbar_init(smem_u32(&b.q_full), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_wait(smem_u32(&b.q_full), 0, &b, err);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s) {
+    wait_timeout_kernel<<<1, 32, 0, s>>>(err);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnParams& p, cudaStream_t s) {

@@ -105,6 +105,61 @@ __global__ void __launch_bounds__(256) euler_kernel(float* __restrict__ x,
     }
 }
 
+// Euler step on the classifier-free-guided velocity (blog chapter 5, "CFG":
+// uncond + w * (cond - uncond)), fused so that the guided velocity is never
+// stored: x += dsigma * (vu + w * (vc - vu)).
+__global__ void __launch_bounds__(256) euler_cfg_kernel(float* __restrict__ x,
+                                                        const float* __restrict__ vc,
+                                                        const float* __restrict__ vu, size_t n,
+                                                        float w, float dsigma) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool vec = ((((uintptr_t)x) | ((uintptr_t)vc) | ((uintptr_t)vu)) & 15) == 0;
+    size_t done = 0;
+    if (vec) {
+        const size_t n4 = n >> 2;
+        float4* x4 = reinterpret_cast<float4*>(x);
+        const float4* c4 = reinterpret_cast<const float4*>(vc);
+        const float4* u4 = reinterpret_cast<const float4*>(vu);
+        for (size_t i = tid; i < n4; i += stride) {
+            float4 a = x4[i];
+            const float4 c = __ldcs(c4 + i), u = __ldcs(u4 + i);
+            a.x = fmaf(dsigma, fmaf(w, c.x - u.x, u.x), a.x);
+            a.y = fmaf(dsigma, fmaf(w, c.y - u.y, u.y), a.y);
+            a.z = fmaf(dsigma, fmaf(w, c.z - u.z, u.z), a.z);
+            a.w = fmaf(dsigma, fmaf(w, c.w - u.w, u.w), a.w);
+            x4[i] = a;
+        }
+        done = n4 << 2;
+    }
+    for (size_t i = done + tid; i < n; i += stride)
+        x[i] = fmaf(dsigma, fmaf(w, vc[i] - vu[i], vu[i]), x[i]);
+}
+
+// Clean-data estimate of flow matching (blog chapter 1): x0 = x - sigma * v.
+__global__ void __launch_bounds__(256) x0_kernel(float* __restrict__ x0,
+                                                 const float* __restrict__ x,
+                                                 const float* __restrict__ v, size_t n,
+                                                 float sigma) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool vec = ((((uintptr_t)x0) | ((uintptr_t)x) | ((uintptr_t)v)) & 15) == 0;
+    size_t done = 0;
+    if (vec) {
+        const size_t n4 = n >> 2;
+        float4* o4 = reinterpret_cast<float4*>(x0);
+        const float4* a4 = reinterpret_cast<const float4*>(x);
+        const float4* v4 = reinterpret_cast<const float4*>(v);
+        for (size_t i = tid; i < n4; i += stride) {
+            const float4 a = __ldcs(a4 + i), b = __ldcs(v4 + i);
+            o4[i] = make_float4(fmaf(-sigma, b.x, a.x), fmaf(-sigma, b.y, a.y),
+                                fmaf(-sigma, b.z, a.z), fmaf(-sigma, b.w, a.w));
+        }
+        done = n4 << 2;
+    }
+    for (size_t i = done + tid; i < n; i += stride) x0[i] = fmaf(-sigma, v[i], x[i]);
+}
+
 int sm_count() {
     static int n = 0;
     if (!n) {
@@ -126,6 +181,22 @@ cudaError_t launch_rope(const RopeParams& p, int max_tok, cudaStream_t s) {
                                                     std::max(1, 8 * sm_count() / p.n_streams));
     dim3 grid(per_stream, p.n_streams);
     rope_append_kernel<<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_euler_cfg(float* x, const float* vc, const float* vu, size_t n, float w,
+                             float dsigma, cudaStream_t s) {
+    const size_t want = (n / 4 + 255) / 256;
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>(want, (size_t)sm_count() * 8));
+    euler_cfg_kernel<<<grid, 256, 0, s>>>(x, vc, vu, n, w, dsigma);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_x0(float* x0, const float* x, const float* v, size_t n, float sigma,
+                      cudaStream_t s) {
+    const size_t want = (n / 4 + 255) / 256;
+    const int grid = (int)std::max<size_t>(1, std::min<size_t>(want, (size_t)sm_count() * 8));
+    x0_kernel<<<grid, 256, 0, s>>>(x0, x, v, n, sigma);
     return cudaGetLastError();
 }
 

@@ -90,8 +90,15 @@ __host__ __device__ inline size_t partial_slot_floats(int D) { return (size_t)kQ
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnParams& p, cudaStream_t s);
 
+// One bounded device wait that runs out (failure-path self-test).
+cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s);
+
 // ----------------------------------------------------------------- Euler
 cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaStream_t s);
+cudaError_t launch_euler_cfg(float* x, const float* vc, const float* vu, size_t n, float w,
+                             float dsigma, cudaStream_t s);
+cudaError_t launch_x0(float* x0, const float* x, const float* v, size_t n, float sigma,
+                      cudaStream_t s);
 
 // ----------------------------------------------------------------- host helpers
 // Encodes a 2D bf16 tensor map over `rows` rows of `D` elements with a

@@ -79,6 +79,13 @@ _SIGS = {
     "pv_euler_step": ([_vp, _vp, _sz, ctypes.c_float, _vp], _i),
     "pv_kv_poll_device_error": ([_vp, ctypes.POINTER(_i)], _i),
     "pv_selftest_exp2_poly": ([_vp, _vp, _sz, _vp], _i),
+    "pv_kv_selftest_wait_timeout": ([_vp, _vp], _i),
+    "pv_attn_varlen_ws_bytes": ([_i, _vp, _vp, _i, _i, ctypes.POINTER(_sz)], _i),
+    "pv_attn_varlen": ([_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
+    "pv_sigma_schedule": ([_i, ctypes.c_double, ctypes.c_double, ctypes.POINTER(ctypes.c_double),
+                           ctypes.POINTER(_i)], _i),
+    "pv_euler_cfg_step": ([_vp, _vp, _vp, _sz, ctypes.c_float, ctypes.c_float, _vp], _i),
+    "pv_x0_estimate": ([_vp, _vp, _vp, _sz, ctypes.c_float, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -207,6 +214,30 @@ def pv_attn_dense(q, k, v, n_q, n_k, heads, head_dim, out, lse, ws, ws_bytes,
                              _ptr(lse), _ptr(ws), ws_bytes, _stream(cuda_stream)))
 
 
+def _lengths(xs):
+    arr = (ctypes.c_int * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+def pv_attn_varlen_ws_bytes(n_q, n_k, heads, head_dim) -> int:
+    """n_q, n_k: per-sequence lengths (host sequences of equal size)."""
+    if len(n_q) != len(n_k):
+        raise ValueError("n_q and n_k differ in length")
+    a = _sz()
+    _check(lib.pv_attn_varlen_ws_bytes(len(n_q), _lengths(n_q), _lengths(n_k), heads, head_dim,
+                                       ctypes.byref(a)))
+    return a.value
+
+
+def pv_attn_varlen(q, k, v, n_q, n_k, heads, head_dim, out, lse, ws, ws_bytes,
+                   cuda_stream=None) -> None:
+    if len(n_q) != len(n_k):
+        raise ValueError("n_q and n_k differ in length")
+    _check(lib.pv_attn_varlen(_ptr(q), _ptr(k), _ptr(v), len(n_q), _lengths(n_q), _lengths(n_k),
+                              heads, head_dim, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
+                              _stream(cuda_stream)))
+
+
 def pv_attn_dense_noalloc(q, k, v, n_q, n_k, heads, head_dim, out, lse=None,
                           cuda_stream=None) -> None:
     _check(lib.pv_attn_dense_noalloc(_ptr(q), _ptr(k), _ptr(v), n_q, n_k, heads, head_dim,
@@ -221,6 +252,29 @@ def pv_kv_poll_device_error(kv) -> int:
     c = _i()
     _check(lib.pv_kv_poll_device_error(kv, ctypes.byref(c)))
     return c.value
+
+
+def pv_sigma_schedule(n_steps, shift, sigma_max=0.0):
+    """(sigmas: list of n_steps + 1 floats, timesteps: list of n_steps ints)."""
+    sig = (ctypes.c_double * (n_steps + 1))()
+    ts = (ctypes.c_int * n_steps)()
+    _check(lib.pv_sigma_schedule(n_steps, shift, sigma_max, sig, ts))
+    return list(sig), list(ts)
+
+
+def pv_euler_cfg_step(x, v_cond, v_uncond, n, guide_scale, dsigma, cuda_stream=None) -> None:
+    _check(lib.pv_euler_cfg_step(_ptr(x), _ptr(v_cond), _ptr(v_uncond), n,
+                                 ctypes.c_float(guide_scale), ctypes.c_float(dsigma),
+                                 _stream(cuda_stream)))
+
+
+def pv_x0_estimate(x0, x, v, n, sigma, cuda_stream=None) -> None:
+    _check(lib.pv_x0_estimate(_ptr(x0), _ptr(x), _ptr(v), n, ctypes.c_float(sigma),
+                              _stream(cuda_stream)))
+
+
+def pv_kv_selftest_wait_timeout(kv, cuda_stream=None) -> None:
+    _check(lib.pv_kv_selftest_wait_timeout(kv, _stream(cuda_stream)))
 
 
 def pv_selftest_exp2_poly(x, y, n, cuda_stream=None) -> None:

@@ -109,3 +109,9 @@ def ragged_fills(n_streams: int, ring_slots: int, seed: int = 0) -> list[int]:
     for i in range(n_streams):
         out.append(_mix32_int(seed_of(0x7F11, seed, i)) % (ring_slots + 1))
     return out
+
+
+def text_lengths(n_prompts: int, max_len: int = 512, seed: int = 0) -> list[int]:
+    """Seeded prompt lengths in 1..max_len, uniform: the real token counts of
+    the text contexts that cross-attention reads (padding trimmed)."""
+    return [1 + _mix32_int(seed_of(0x7E47, seed, i)) % max_len for i in range(n_prompts)]

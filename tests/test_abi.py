@@ -177,3 +177,52 @@ def test_row_offsets_follow_the_documented_layout():
     with pytest.raises(pv.PVError):
         pv.pv_kv_row_offset(h, 2, 0, 0, 0, 0)
     pv.pv_kv_destroy(h)
+
+
+# ------------------------------------------------------------------ sampler schedule (host)
+from oracle import euler  # noqa: E402
+from golden_io import load as read_golden  # noqa: E402
+
+
+@pytest.mark.parametrize("n,shift", [(1, 1.0), (4, 1.0), (4, 5.0), (40, 12.0), (50, 3.0),
+                                     (1000, 12.0)])
+def test_sigma_schedule_matches_oracle(n, shift):
+    sig, ts = pv.pv_sigma_schedule(n, shift)
+    ref = euler.shifted_schedule(n, shift)
+    assert len(sig) == n + 1 and sig[-1] == 0.0
+    for a, b in zip(sig, ref):
+        assert abs(a - b) <= 4e-16 * max(1.0, abs(b))
+    assert ts == list(euler.timesteps(ref[:-1]))
+
+
+def test_sigma_schedule_printed_timesteps():
+    g = read_golden("shift_schedule.txt")
+    sig, ts = pv.pv_sigma_schedule(int(g["steps"]), float(g["shift"]))
+    assert ts[:6] == [int(g[f"t{i}"]) for i in range(6)]
+    assert sum(t >= int(g["high_noise_boundary"]) for t in ts) == int(g["steps_at_or_above_boundary"])
+
+
+def test_sigma_schedule_explicit_top_and_errors():
+    sig, ts = pv.pv_sigma_schedule(4, 1.0, 1.0)
+    assert sig == [1.0, 0.75, 0.5, 0.25, 0.0]      # the plain four-step grid
+    assert ts == [1000, 750, 500, 250]
+    for args in [(0, 1.0), (4, 0.0), (4, -2.0), (4, float("nan")), (4, 1.0, 1.5)]:
+        with pytest.raises(pv.PVError) as e:
+            pv.pv_sigma_schedule(*args)
+        assert e.value.status == pv.PV_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ varlen attention (host checks)
+def test_varlen_workspace_and_shape_checks():
+    one = pv.pv_attn_varlen_ws_bytes([880], [512], 24, 128)
+    dense = pv.pv_attn_dense_ws_bytes(880, 512, 24, 128)
+    assert one == dense and one % 256 == 0
+    batch = pv.pv_attn_varlen_ws_bytes([2640, 880, 0, 880], [77, 512, 0, 1], 24, 128)
+    assert batch > one
+    for n_q, n_k, D in (([5], [0], 128), ([-1], [3], 128), ([1] * 65, [1] * 65, 128),
+                        ([4], [4], 96)):
+        with pytest.raises(pv.PVError) as e:
+            pv.pv_attn_varlen_ws_bytes(n_q, n_k, 2, D)
+        assert e.value.status == pv.PV_ERR_SHAPE
+    # no queries anywhere: a no-op that touches no device
+    pv.pv_attn_varlen(0, 0, 0, [0, 0], [3, 0], 2, 64, 0, None, 0, 0)

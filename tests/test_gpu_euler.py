@@ -77,3 +77,75 @@ def test_exp2_polynomial_against_exp2(pv):
     rel_cuda = (torch.abs(y[main] - ref_cuda[main]) / ref_cuda[main]).max().item()
     assert rel64.max() <= 1e-4 and rel_cuda <= 1e-4, (rel64.max(), rel_cuda)
     assert torch.all(y[-4:] <= 2.0 ** -124) and torch.all(y[-4:] > 0)
+
+
+# ------------------------------------------------------------------ sampler variants
+@pytest.mark.parametrize("n,offset,w", [(1, 0, 5.0), (13, 1, 5.0), (FRAME + 3, 1, 4.0),
+                                        (31 * FRAME, 0, 5.0), (31 * FRAME, 0, 1.0),
+                                        (31 * FRAME, 0, 0.0)])
+def test_euler_cfg_step_matches_oracle(pv, n, offset, w):
+    x = synth.normal_f32(111, (n + offset,), "cuda")
+    vc = synth.normal_f32(112, (n + offset,), "cuda")
+    vu = synth.normal_f32(113, (n + offset,), "cuda")
+    xh, ch, uh = f64(x)[offset:], f64(vc)[offset:], f64(vu)[offset:]
+    sig = euler.shifted_schedule(40, 12.0)
+    for i in (0, 17, 39):
+        ref = euler.euler_cfg_step(xh, ch, uh, w, sig[i], sig[i + 1])
+        d = float(sig[i + 1] - sig[i])
+        pv.pv_euler_cfg_step(x[offset:], vc[offset:], vu[offset:], n, w, d)
+        torch.cuda.synchronize()
+        got = f64(x)[offset:]
+        # f32 terms: |x|, |d| (|vu| + |w| (|vc| + |vu|)), each a few ulps
+        bound = 2e-6 * (np.abs(xh) + abs(d) * (np.abs(uh) + abs(w) * (np.abs(ch) + np.abs(uh))))
+        assert np.all(np.abs(got - ref) <= bound + 1e-30)
+        xh = ref
+    if offset:
+        assert float(x[0]) == float(synth.normal_f32(111, (1,))[0])
+
+
+def test_euler_cfg_special_cases(pv):
+    n = 2 * FRAME
+    x = synth.normal_f32(114, (n,), "cuda")
+    vc = synth.normal_f32(115, (n,), "cuda")
+    vu = synth.normal_f32(116, (n,), "cuda")
+    # w = 1 is the conditional step, w = 0 the unconditional one
+    for w, v in ((1.0, vc), (0.0, vu)):
+        a, b = x.clone(), x.clone()
+        pv.pv_euler_cfg_step(a, vc, vu, n, w, -0.125)
+        pv.pv_euler_step(b, v, n, -0.125)
+        torch.cuda.synchronize()
+        assert torch.max(torch.abs(a - b)).item() <= 1e-6 * torch.max(torch.abs(b)).item()
+    # equal velocities: guidance has nothing to amplify
+    a, b = x.clone(), x.clone()
+    pv.pv_euler_cfg_step(a, vc, vc, n, 5.0, -0.125)
+    pv.pv_euler_step(b, vc, n, -0.125)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    with pytest.raises(pv.PVError):
+        pv.pv_euler_cfg_step(x, vc, 0, n, 5.0, -0.1)
+    with pytest.raises(pv.PVError):
+        pv.pv_euler_cfg_step(x, vc, vu, n, float("inf"), -0.1)
+
+
+@pytest.mark.parametrize("n,offset", [(1, 0), (9, 1), (FRAME + 1, 1), (31 * FRAME, 0)])
+def test_x0_estimate_matches_oracle(pv, n, offset):
+    x = synth.normal_f32(121, (n + offset,), "cuda")
+    v = synth.normal_f32(122, (n + offset,), "cuda")
+    out = torch.full((n + offset,), 7.0, device="cuda")
+    xh, vh = f64(x)[offset:], f64(v)[offset:]
+    for sigma in (1.0, 0.75, 0.3125, 0.0):
+        pv.pv_x0_estimate(out[offset:], x[offset:], v[offset:], n, sigma)
+        torch.cuda.synchronize()
+        ref = euler.x0_prediction(xh, vh, sigma)
+        got = f64(out)[offset:]
+        assert np.all(np.abs(got - ref) <= 2**-23 * (np.abs(xh) + sigma * np.abs(vh)) + 1e-30)
+    if offset:
+        assert float(out[0]) == 7.0
+    # in place (x0 aliases x), and the straight line: x = (1-s) x0 + s x1, v = x1 - x0
+    x0 = synth.normal_f32(123, (n,), "cuda")
+    x1 = synth.normal_f32(124, (n,), "cuda")
+    s = 0.375
+    xs = (1 - s) * x0 + s * x1
+    pv.pv_x0_estimate(xs, xs, x1 - x0, n, s)
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(xs - x0)).item() <= 4e-6 * torch.max(torch.abs(x0) + torch.abs(x1)).item()
