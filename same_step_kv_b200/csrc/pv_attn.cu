@@ -547,6 +547,92 @@ __device__ __forceinline__ float row_max(const uint32_t* sr) {
                  fmaxf(mx8[6], mx8[7]));
 }
 
+// Normalised bf16 output of 32 f32 columns: row dst[0..32) = o * inv.
+__device__ __forceinline__ void store_row32(bf16* dst, const uint32_t* o, float inv) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int q = i * 8;
+        d4[i] = make_uint4(
+            pack_bf16(__uint_as_float(o[q + 0]) * inv, __uint_as_float(o[q + 1]) * inv),
+            pack_bf16(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv),
+            pack_bf16(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv),
+            pack_bf16(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv));
+    }
+}
+
+// Merge of the split parts of one query tile by the last CTA to arrive
+// (split-KV combination of the online softmax: with M = max_k m_k and
+// L = sum_k l_k 2^(m_k - M), o = sum_k O_k 2^(m_k - M) / L).  Part k sits in
+// the partial slot of CTA c_first + k; with `keep` this CTA's own part is
+// still in TMEM (tO, m_own, l_own) and is taken from there, bit for bit the
+// values it stored.  Sums run in part order whichever CTA merges, so results
+// are reproducible.  The (m, l) loads are issued four parts at a time and a
+// part's 32-column block in one batch: a merge costs a few L2 round trips.
+template <int D>
+__device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, int X, int r,
+                                            bool row_ok, bool keep, uint32_t tO, float m_own,
+                                            float l_own, bf16* dst, float* lse_dst) {
+    const size_t slot_f = partial_slot_floats(D);
+    const int self = keep ? (int)blockIdx.x - g.c_first : -1;
+    auto ml = [&](int k) -> const float* {
+        return p.partial + part_slot(p, g.c_first + k, g.i0, X) * slot_f + (size_t)kQRows * D;
+    };
+    float M = -INFINITY;
+    for (int k0 = 0; k0 < g.nseg; k0 += 4) {
+        float mk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u;
+            mk[u] = k == self ? m_own : (k < g.nseg ? __ldcg(ml(k) + r) : -INFINITY);
+        }
+        M = fmaxf(fmaxf(M, fmaxf(mk[0], mk[1])), fmaxf(mk[2], mk[3]));
+    }
+    float L = 0.f;
+    for (int k0 = 0; k0 < g.nseg; k0 += 4) {
+        float mk[4], lk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u;
+            mk[u] = k == self ? m_own : (k < g.nseg ? __ldcg(ml(k) + r) : 0.f);
+            lk[u] = k == self ? l_own : (k < g.nseg ? __ldcg(ml(k) + kQRows + r) : 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (k0 + u < g.nseg) L += lk[u] * ex2(mk[u] - M);
+    }
+    const float invL = 1.0f / L;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        for (int k = 0; k < g.nseg; ++k) {
+            uint32_t v[32];
+            float w;
+            if (k == self) {
+                tmem_ld32_wait(tO + c, v);
+                w = ex2(m_own - M) * invL;
+            } else {
+                const float* pk = ml(k) - (size_t)kQRows * D;
+                w = ex2(__ldcg(pk + (size_t)kQRows * D + r) - M) * invL;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = __float_as_uint(__ldcg(pk + (size_t)(c + i) * kQRows + r));
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __uint_as_float(v[i]), acc[i]);
+        }
+        if (row_ok) {
+            uint32_t o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(acc[i]);
+            store_row32(dst + c, o, 1.0f);
+        }
+    }
+    if (row_ok && lse_dst) *lse_dst = (M + __log2f(L)) * 0.69314718055994531f;
+}
+
 template <int D>
 __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, int X) {
     using C = Cfg<D>;
@@ -623,41 +709,36 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         // ------------------------------------------------------ epilogue
         const bool row_ok = r < g.rows[X];
         const int tok = s.out_tok0 + g.q0 + X * kQRows + r;
-        // O leaves TMEM in 32-column chunks: to the output when this CTA
-        // holds the whole item, else to this CTA's partial slot.
         const bool whole = g.nseg == 1;
+        // On the CTA's last segment O may stay in TMEM until the arrival
+        // count says whether this CTA merges: the merge then reads its own
+        // part from there instead of back from global memory.
+        const bool keep = !whole && it.pos >= it.end;
         const float inv = 1.0f / l;
         bf16* dst = p.out + ((size_t)tok * p.heads + g.head) * D;
         float* mine = p.partial + part_slot(p, blockIdx.x, g.i0, X) * slot_f;
+        // O leaves TMEM in 32-column chunks: to the output when this CTA
+        // holds the whole item, else to this CTA's partial slot
+        // (column-major [D][128], then m[128], l[128]: a warp stores 32
+        // consecutive floats).
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
             tmem_ld32_wait(tO + c, o);
             if (whole) {
-                if (row_ok) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int q = i * 8;
-                        d4[i] = make_uint4(
-                            pack_bf16(__uint_as_float(o[q + 0]) * inv, __uint_as_float(o[q + 1]) * inv),
-                            pack_bf16(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv),
-                            pack_bf16(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv),
-                            pack_bf16(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv));
-                    }
-                }
+                if (row_ok) store_row32(dst + c, o, inv);
             } else {
-                // column-major slot ([D][128], m[128], l[128]): a warp stores 32
-                // consecutive floats
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     __stcg(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]));
             }
         }
-        // O is read out: the next segment's first P V may overwrite it
-        tc_fence_before();
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->o_empty[X]));
+        if (!keep) {
+            // O is read out: the next segment's first P V may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->o_empty[X]));
+        }
         if (whole) {
             if (row_ok && p.lse) p.lse[(size_t)tok * p.heads + g.head] = (m + __log2f(l)) * ln2;
             continue;
@@ -684,43 +765,16 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         }
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->ep_out[X]), ec & 1, b, p.err));
         ++ec;
-        if (!ok) break;
-        if (!b->last[X] || !row_ok) continue;
-        __threadfence();
-        // the parts of this item: CTAs c_first .. c_first + nseg - 1
-        const long long i0 = g.i0;
-        float M = -INFINITY;
-        for (int k = 0; k < g.nseg; ++k) {
-            const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
-            M = fmaxf(M, __ldcg(pk + (size_t)kQRows * D + r));
+        if (ok && b->last[X]) {
+            __threadfence();
+            merge_parts<D>(p, g, X, r, row_ok, keep, tO, m, l, dst,
+                           p.lse ? p.lse + (size_t)tok * p.heads + g.head : nullptr);
         }
-        float L = 0.f;
-        for (int k = 0; k < g.nseg; ++k) {
-            const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
-            L += __ldcg(pk + (size_t)kQRows * D + kQRows + r) * ex2(__ldcg(pk + (size_t)kQRows * D + r) - M);
+        if (keep) {
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->o_empty[X]));
         }
-        const float invL = 1.0f / L;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-            float acc[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-            for (int k = 0; k < g.nseg; ++k) {
-                const float* pk = p.partial + part_slot(p, g.c_first + k, i0, X) * slot_f;
-                const float w = ex2(__ldcg(pk + (size_t)kQRows * D + r) - M) * invL;
-                float v[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) v[q] = __ldcg(pk + (size_t)(c + q) * kQRows + r);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) acc[q] = fmaf(w, v[q], acc[q]);
-            }
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-            d4[0] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
-                               pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
-            d4[1] = make_uint4(pack_bf16(acc[8], acc[9]), pack_bf16(acc[10], acc[11]),
-                               pack_bf16(acc[12], acc[13]), pack_bf16(acc[14], acc[15]));
-        }
-        if (p.lse) p.lse[(size_t)tok * p.heads + g.head] = (M + __log2f(L)) * ln2;
     }
 }
 
