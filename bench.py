@@ -11,6 +11,7 @@ every layer is pre-filled, and the working set (6.9 GB of K/V) is far larger
 than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload step|cross_attn|sampler]
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 on the host cores on a bounded sample of the same workload.
@@ -93,6 +94,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # nvidia-smi takes a moment to start: let sampling be live before
+            # the timed region begins
+            t_end = time.time() + 3.0
+            while not self.lines and time.time() < t_end:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
@@ -177,16 +183,222 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def timed_steps(step, args, local, world, cs):
+    """W untimed steps, then K steps between CUDA events on `cs`, with clocks
+    sampled meanwhile.  Returns (ms per step, max over ranks; clock summary)."""
+    import torch
+    import torch.distributed as dist
+    from same_step_kv_b200.dist import max_over_ranks
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(cs)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(cs)
+        torch.cuda.synchronize()
+    return max_over_ranks(t0.elapsed_time(t1)) / args.steps, clk.summary()
+
+
+def bound_roofline(flops, nbytes, seconds, peaks, src, kernel):
+    """Roofline object for a kernel that may be bound by either pipe: the bound
+    is whichever of flops / tensor peak and bytes / HBM peak takes longer."""
+    tensor_peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    hbm_peak = float(peaks["hbm_gbs"])
+    if flops / (tensor_peak * 1e12) >= nbytes / (hbm_peak * 1e9):
+        a = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": a / tensor_peak, "peak_source": f"{src} bf16_tflops_sustained",
+                "kernel": kernel, "traffic": None,
+                "hbm_achieved_gbs": nbytes / seconds / 1e9}
+    a = nbytes / seconds / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": hbm_peak, "unit": "GB/s", "frac": a / hbm_peak,
+            "peak_source": f"{src} hbm_gbs", "kernel": kernel, "traffic": None,
+            "tensor_achieved_tflops": flops / seconds / 1e12}
+
+
+N_PROMPTS = 8       # cross-attention: prompts served together, one latent frame each
+MAX_TEXT = 512      # longest text context (tokens)
+
+
+def run_cross_attn(args, rank, world, local):
+    """Cross-attention of N_PROMPTS prompts, each one latent frame (880 video
+    tokens) querying its own text context of 1..512 tokens, 24 x 128, one
+    pv_attn_varlen launch per layer, 30 layers per step."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    NL = args.layers
+    n_k = synth.text_lengths(N_PROMPTS, MAX_TEXT, seed=rank)
+    n_q = [T] * N_PROMPTS
+    tq, tk = sum(n_q), sum(n_k)
+    q = [synth.normal_bf16(synth.seed_of(0x5101, rank, l), (HEADS * tq * D,), dev) for l in range(NL)]
+    k = [synth.normal_bf16(synth.seed_of(0x5102, rank, l), (HEADS * tk * D,), dev) for l in range(NL)]
+    v = [synth.normal_bf16(synth.seed_of(0x5103, rank, l), (HEADS * tk * D,), dev) for l in range(NL)]
+    out = torch.empty(tq, HEADS, D, dtype=torch.bfloat16, device=dev)
+    wsb = pv.pv_attn_varlen_ws_bytes(n_q, n_k, HEADS, D)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    ev = []
+
+    def step(record):
+        for l in range(NL):
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+            pv.pv_attn_varlen(q[l], k[l], v[l], n_q, n_k, HEADS, D, out, None, ws, wsb, cs)
+            if record:
+                e1.record(cs)
+                ev.append((e0, e1))
+
+    ms_step, clocks = timed_steps(step, args, local, world, cs)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = sum(4 * a * b * HEADS * D for a, b in zip(n_q, n_k))
+    nbytes = (2 * tq + 2 * tk) * HEADS * D * 2          # q, out; k, v
+    # e2e: each layer's q and text context from pinned host memory, output read back
+    hq = [t.cpu().pin_memory() for t in q]
+    hk = [t.cpu().pin_memory() for t in k]
+    hv = [t.cpu().pin_memory() for t in v]
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q[0]), torch.empty_like(k[0]), torch.empty_like(v[0])
+
+    def e2e_step(record):
+        for l in range(NL):
+            dq.copy_(hq[l], non_blocking=True)
+            dk.copy_(hk[l], non_blocking=True)
+            dv.copy_(hv[l], non_blocking=True)
+            pv.pv_attn_varlen(dq, dk, dv, n_q, n_k, HEADS, D, out, None, ws, wsb, cs)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    if rank == 0:
+        peaks, src = load_peaks()
+        line = {
+            "metric": "cross-attention TFLOP/s (30 layers x 8 prompts, one launch per layer)",
+            "value": NL * flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"cross-attention, {N_PROMPTS} prompts x 880 video tokens, "
+                                   f"text 1..{MAX_TEXT} tokens, 24x128, {NL} layers",
+                       "text_lengths": n_k,
+                       "l2": f"inputs larger than L2 ({NL * (tq + 2 * tk) * HEADS * D * 2 / 1e9:.2f} GB "
+                             "per step), no flush"},
+            "roofline": bound_roofline(flops, nbytes, launch_ms * 1e-3, peaks, src,
+                                       "attn_kernel<128> (pv_attn_varlen)"),
+            "e2e": {"value": NL * flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": NL * (tq + 2 * tk) * HEADS * D * 2,
+                    "d2h_bytes_per_step": tq * HEADS * D * 2},
+            "gpu_launches": args.steps * NL, "clocks": clocks, "cpu_baseline": None,
+        }
+        line["roofline"]["ms_per_launch"] = launch_ms
+        print(json.dumps(line), flush=True)
+
+
+SAMPLER_FRAMES = 248   # 8 streams x 31 latent frames
+
+
+def run_sampler(args, rank, world, local):
+    """One sampler step over a batch of SAMPLER_FRAMES latent frames (48 x 44 x 80
+    each): the CFG-guided Euler update (x, v_cond, v_uncond in, x out: 16 B per
+    value) and the x0 estimate (x, v in, x0 out: 12 B per value)."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    n = SAMPLER_FRAMES * LATENT
+    x = synth.normal_f32(synth.seed_of(0x5A01, rank), (n,), dev)
+    vc = synth.normal_f32(synth.seed_of(0x5A02, rank), (n,), dev)
+    vu = synth.normal_f32(synth.seed_of(0x5A03, rank), (n,), dev)
+    x0 = torch.empty_like(x)
+    sig = pv.pv_sigma_schedule(40, 12.0)[0]
+    d = float(sig[21] - sig[20])
+    w = 5.0
+    ev = []
+
+    def step(record):
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(cs)
+        pv.pv_euler_cfg_step(x, vc, vu, n, w, d, cs)
+        if record:
+            e1.record(cs)
+            ev.append((e0, e1))
+        pv.pv_x0_estimate(x0, x, vc, n, float(sig[21]), cs)
+
+    ms_step, clocks = timed_steps(step, args, local, world, cs)
+    cfg_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    step_bytes = 16 * n + 12 * n
+    # e2e: velocities in from pinned host memory, x0 read back
+    hvc, hvu = vc.cpu().pin_memory(), vu.cpu().pin_memory()
+    hx0 = torch.empty(n, dtype=torch.float32).pin_memory()
+
+    def e2e_step(record):
+        vc.copy_(hvc, non_blocking=True)
+        vu.copy_(hvu, non_blocking=True)
+        pv.pv_euler_cfg_step(x, vc, vu, n, w, d, cs)
+        pv.pv_x0_estimate(x0, x, vc, n, float(sig[21]), cs)
+        hx0.copy_(x0, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    if rank == 0:
+        peaks, src = load_peaks()
+        hbm = float(peaks["hbm_gbs"])
+        a = 16 * n / (cfg_ms * 1e-3) / 1e9
+        line = {
+            "metric": "sampler GB/s (CFG-guided Euler step + x0 estimate)",
+            "value": step_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"sampler, {SAMPLER_FRAMES} latent frames of 48x44x80 "
+                                   "(shift 12, step 20 of 40, guide scale 5)",
+                       "values": n, "l2": f"inputs larger than L2 ({4 * n * 4 / 1e9:.2f} GB), no flush"},
+            "roofline": {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+                         "peak_source": f"{src} hbm_gbs", "kernel": "euler_cfg_kernel",
+                         "ms_per_launch": cfg_ms, "traffic": None},
+            "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": 8 * n, "d2h_bytes_per_step": 4 * n},
+            "gpu_launches": 2 * args.steps, "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 100 for step, 400 for cross_attn, 2000 for sampler)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers per step (30 in the profile; fewer only for small ncu captures)")
+    ap.add_argument("--workload", default="step", choices=["step", "cross_attn", "sampler"],
+                    help="step: the same-step KV chunk step (default); cross_attn, sampler: "
+                         "the cross-attention and sampler-variant kernels on their own")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = {"step": 100, "cross_attn": 400, "sampler": 2000}[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -195,6 +407,12 @@ def main():
     NL = args.layers
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.workload != "step":
+        (run_cross_attn if args.workload == "cross_attn" else run_sampler)(args, rank, world, local)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
 
     import torch

@@ -273,8 +273,10 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 // (see pv_plan.cu).  A segment is the part of one item inside that range.
 __device__ __forceinline__ long long bound(const AttnParams& p, int c) {
     if (!p.item_aligned) return (long long)c * p.total / p.grid;
-    // whole items: CTA c starts at item c * n_items / grid
-    const int k = (int)((long long)c * p.n_items / p.grid);
+    // whole items: CTA c starts at item first_item[c] (balanced by the host),
+    // or at item c * n_items / grid when the table cannot hold the indices
+    const int k = p.item_aligned == 1 ? (int)p.first_item[c]
+                                      : (int)((long long)c * p.n_items / p.grid);
     int i = 0;
     while (i + 1 < p.n_streams && p.st[i + 1].item0 <= k) ++i;
     if (k >= p.n_items) return p.total;
@@ -874,6 +876,9 @@ cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s) {
     wait_timeout_kernel<<<1, 32, 0, s>>>(err);
     return cudaGetLastError();
 }
+
+static_assert(sizeof(AttnParams) + 3 * sizeof(CUtensorMap) <= 4096,
+              "attention kernel parameters beyond 4 KB");
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnParams& p, cudaStream_t s) {

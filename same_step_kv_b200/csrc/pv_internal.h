@@ -64,9 +64,10 @@ struct AttnStreamDesc {
     long long cost0;     // key tiles of all items before this stream's first
 };
 
-// One launch is a stream-K schedule: the items (head, query block) of all
-// streams, in order, each costing n_kt key tiles, laid end to end; CTA c
-// of `grid` processes the key tiles [c*total/grid, (c+1)*total/grid).
+// One launch is a list of items (head, query block) of all streams, each
+// costing n_kt key tiles, laid end to end; CTA c of `grid` processes one
+// contiguous range of that list (pv_plan.cu chooses the ranges).  The whole
+// struct plus three tensor maps stays under 4 KB of kernel parameters.
 struct AttnParams {
     bf16* out;
     float* lse;
@@ -78,9 +79,11 @@ struct AttnParams {
     float scale_log2;    // log2(e) / sqrt(D)
     int n_streams;
     int grid;            // CTAs of the launch
-    int item_aligned;    // 1: CTA ranges end on item boundaries (no partial results)
+    int item_aligned;    // 0: stream-K; 1, 2: CTA ranges end on item boundaries (no partial
+                         // results), at first_item[] (1) or at equal item counts (2)
     int n_items;         // items of all streams
     long long total;     // key tiles of all items
+    uint16_t first_item[kMaxGrid + 1];  // item_aligned == 1: CTA c's first item
     AttnStreamDesc st[PV_MAX_STREAMS];
 };
 
