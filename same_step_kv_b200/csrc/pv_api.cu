@@ -170,6 +170,31 @@ bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, 
     return true;
 }
 
+// The attention output out[token][head][D] (bf16) as a 3D tensor (D, heads,
+// tokens) for TMA stores: a box is 64 columns of one head for 32 consecutive
+// tokens (one softmax warp's rows), 128-byte swizzled like the staging buffer.
+bool encode_out_map(CUtensorMap* map, void* out, long long tokens, int heads, int D, char* err,
+                    size_t errlen) {
+    auto enc = get_encode();
+    if (!enc) {
+        snprintf(err, errlen, "cuTensorMapEncodeTiled is not available from the driver");
+        return false;
+    }
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)D * sizeof(bf16), (cuuint64_t)heads * D * sizeof(bf16)};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kOutRows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(err, errlen, "cuTensorMapEncodeTiled failed (%d) for the output, %lld tokens x %d x %d",
+                 (int)r, tokens, heads, D);
+        return false;
+    }
+    return true;
+}
+
 }  // namespace pv
 
 struct pv_kv_s {
@@ -188,6 +213,10 @@ struct pv_kv_s {
     // cached tensor map of the last q_rot buffer
     const void* qmap_ptr = nullptr;
     long long qmap_rows = -1;
+    // cached tensor map of the last output buffer
+    CUtensorMap tm_o{};
+    const void* omap_ptr = nullptr;
+    long long omap_rows = -1;
     CUtensorMap tm_q{};
 };
 
@@ -252,6 +281,18 @@ pv_status q_map(pv_kv kv, const void* q_rot, long long rows, CUtensorMap* out) {
         kv->qmap_rows = rows;
     }
     *out = kv->tm_q;
+    return PV_OK;
+}
+
+pv_status out_map(pv_kv kv, void* out, long long tokens, CUtensorMap* map) {
+    if (out != kv->omap_ptr || tokens != kv->omap_rows) {
+        char msg[256];
+        if (!encode_out_map(&kv->tm_o, out, tokens, kv->cfg.heads, kv->cfg.head_dim, msg, sizeof msg))
+            return fail(PV_ERR_CUDA, "%s", msg);
+        kv->omap_ptr = out;
+        kv->omap_rows = tokens;
+    }
+    *map = kv->tm_o;
     return PV_OK;
 }
 
@@ -609,9 +650,10 @@ pv_status pv_chunk_attn(pv_kv kv, int n_streams, const int* streams, int layer, 
     }
     if (plan_attention(p, kv->n_sm, kv->wl.n_partials, kv->wl.n_counters) < 0)
         return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
-    CUtensorMap tq;
+    CUtensorMap tq, to;
     if ((st = q_map(kv, q_rot, (long long)c.heads * tok, &tq))) return st;
-    cudaError_t e = launch_attn(tq, kv->tm_k, kv->tm_v, p, (cudaStream_t)cuda_stream);
+    if ((st = out_map(kv, out, tok, &to))) return st;
+    cudaError_t e = launch_attn(tq, kv->tm_k, kv->tm_v, to, p, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "chunk_attn launch");
     return PV_OK;
 }
@@ -721,11 +763,13 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
         return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
     CUtensorMap tq, tk, tv;
     char msg[256];
+    CUtensorMap to;
     if (!encode_rows_map(&tq, q, (long long)heads * n_q, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tk, k, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
-        !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg))
+        !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
+        !encode_out_map(&to, out, n_q, heads, head_dim, msg, sizeof msg))
         return fail(PV_ERR_CUDA, "%s", msg);
-    cudaError_t e = launch_attn(tq, tk, tv, p, (cudaStream_t)cuda_stream);
+    cudaError_t e = launch_attn(tq, tk, tv, to, p, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_dense launch");
     return PV_OK;
 }
@@ -794,11 +838,13 @@ pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs
         return fail(PV_ERR_CAPACITY, "attention plan exceeds the workspace");
     CUtensorMap tq, tk, tv;
     char msg[256];
+    CUtensorMap to;
     if (!encode_rows_map(&tq, q, heads * tot_q, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tk, k, heads * tot_k, head_dim, msg, sizeof msg) ||
-        !encode_rows_map(&tv, v, heads * tot_k, head_dim, msg, sizeof msg))
+        !encode_rows_map(&tv, v, heads * tot_k, head_dim, msg, sizeof msg) ||
+        !encode_out_map(&to, out, tot_q, heads, head_dim, msg, sizeof msg))
         return fail(PV_ERR_CUDA, "%s", msg);
-    cudaError_t e = launch_attn(tq, tk, tv, p, (cudaStream_t)cuda_stream);
+    cudaError_t e = launch_attn(tq, tk, tv, to, p, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "attn_varlen launch");
     return PV_OK;
 }

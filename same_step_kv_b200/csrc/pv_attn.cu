@@ -44,10 +44,13 @@ template <int D>
 struct Cfg {
     static constexpr int kSub = D / 64;                      // 64-column swizzle sub-tiles
     static constexpr int kTileBytes = kQRows * D * 2;        // one 128-row tile
-    static constexpr int kStages = D == 128 ? 5 : 8;         // K/V ring depth
+    static constexpr int kStages = D == 128 ? 4 : 8;         // K/V ring depth
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
-    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    // output staging: 32 rows x 64 columns of bf16 (4 KB) per softmax warp
+    static constexpr int kEpiOff = kKVOff + kStages * kTileBytes;
+    static constexpr int kEpiWarpBytes = kOutRows * 64 * 2;
+    static constexpr int kBarOff = kEpiOff + 8 * kEpiWarpBytes;
     static constexpr int kSmem = kBarOff + 512 + 1024;       // + barriers + alignment slack
     static constexpr uint32_t kColsO = 256;
 };
@@ -157,6 +160,30 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, i
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+
+// TMA store of the box at (c0, c1, c2) of a 3D tensor map from shared memory,
+// in this thread's bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(src)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Make this thread's shared-memory writes visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05
@@ -563,6 +590,41 @@ __device__ __forceinline__ void store_row32(bf16* dst, const uint32_t* o, float 
     }
 }
 
+// Coalesced output.  One thread holds one query row, and rows of one head are
+// 6 KB apart in out[token][head][D], so direct stores touch 32 cache lines per
+// warp instruction.  Instead a warp whose 32 rows are all queries puts its
+// rows into its own shared-memory buffer (32 rows x 64 columns of bf16, the
+// 16-byte chunk k of row r at chunk k ^ (r & 7): the 128-byte swizzle of the
+// output tensor map, and free of bank conflicts) and one TMA store writes the
+// block as whole 128-byte row pieces.
+// Columns 32h .. 32h+31 of the staged 64-column block, scaled by `scale`.
+__device__ __forceinline__ void stage_put32(uint8_t* buf, int h, const uint32_t* o, float scale) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int q = i * 8;
+        const int k = h * 4 + i;
+        *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = make_uint4(
+            pack_bf16(__uint_as_float(o[q + 0]) * scale, __uint_as_float(o[q + 1]) * scale),
+            pack_bf16(__uint_as_float(o[q + 2]) * scale, __uint_as_float(o[q + 3]) * scale),
+            pack_bf16(__uint_as_float(o[q + 4]) * scale, __uint_as_float(o[q + 5]) * scale),
+            pack_bf16(__uint_as_float(o[q + 6]) * scale, __uint_as_float(o[q + 7]) * scale));
+    }
+}
+// Before the buffer is written again: the warp's previous store has read it.
+__device__ __forceinline__ void stage_acquire() {
+    if ((threadIdx.x & 31) == 0) bulk_wait_read();
+    __syncwarp();
+}
+// The staged block to out: columns c0 .. c0+63 of `head` for tokens tok0 ..
+// tok0+31, one TMA store issued by lane 0.
+__device__ __forceinline__ void stage_flush(const CUtensorMap* to, const uint8_t* buf, int c0,
+                                            int head, int tok0) {
+    fence_async_smem();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tma_store_3d(to, smem_u32(buf), c0, head, tok0);
+}
+
 // Merge of the split parts of one query tile by the last CTA to arrive
 // (split-KV combination of the online softmax: with M = max_k m_k and
 // L = sum_k l_k 2^(m_k - M), o = sum_k O_k 2^(m_k - M) / L).  Part k sits in
@@ -574,7 +636,9 @@ __device__ __forceinline__ void store_row32(bf16* dst, const uint32_t* o, float 
 template <int D>
 __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, int X, int r,
                                             bool row_ok, bool keep, uint32_t tO, float m_own,
-                                            float l_own, bf16* dst, float* lse_dst) {
+                                            float l_own, bf16* dst, float* lse_dst,
+                                            const CUtensorMap* to, uint8_t* ebuf, bool warp_full,
+                                            int tok_w) {
     const size_t slot_f = partial_slot_floats(D);
     const int self = keep ? (int)blockIdx.x - g.c_first : -1;
     auto ml = [&](int k) -> const float* {
@@ -625,10 +689,14 @@ __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, i
 #pragma unroll
             for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, __uint_as_float(v[i]), acc[i]);
         }
-        if (row_ok) {
-            uint32_t o[32];
+        uint32_t o[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(acc[i]);
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(acc[i]);
+        if (warp_full) {
+            if ((c & 63) == 0) stage_acquire();
+            stage_put32(ebuf, (c >> 5) & 1, o, 1.0f);
+            if ((c & 63) == 32) stage_flush(to, ebuf, c - 32, g.head, tok_w);
+        } else if (row_ok) {
             store_row32(dst + c, o, 1.0f);
         }
     }
@@ -636,13 +704,15 @@ __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, i
 }
 
 template <int D>
-__device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, int X) {
+__device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uint8_t* smem,
+                                 Bars* b, uint32_t tmem, int X) {
     using C = Cfg<D>;
     const int wq = (threadIdx.x / 32) & 3;          // TMEM lane quadrant of this warp
     const int r = wq * 32 + (threadIdx.x & 31);     // query row inside the tile
     const uint32_t lane = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane + X * 128;
     const uint32_t tO = tmem + lane + C::kColsO + X * D;
+    uint8_t* ebuf = smem + C::kEpiOff + (X * 4 + wq) * C::kEpiWarpBytes;  // this warp's staging
     const float sl2 = p.scale_log2;
     const float ln2 = 0.69314718055994531f;
     const size_t slot_f = partial_slot_floats(D);
@@ -719,6 +789,8 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         const float inv = 1.0f / l;
         bf16* dst = p.out + ((size_t)tok * p.heads + g.head) * D;
         float* mine = p.partial + part_slot(p, blockIdx.x, g.i0, X) * slot_f;
+        const bool warp_full = wq * 32 + 31 < g.rows[X];  // all 32 rows of this warp are queries
+        const int tok_w = s.out_tok0 + g.q0 + X * kQRows + wq * 32;
         // O leaves TMEM in 32-column chunks: to the output when this CTA
         // holds the whole item, else to this CTA's partial slot
         // (column-major [D][128], then m[128], l[128]: a warp stores 32
@@ -728,7 +800,13 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
             uint32_t o[32];
             tmem_ld32_wait(tO + c, o);
             if (whole) {
-                if (row_ok) store_row32(dst + c, o, inv);
+                if (warp_full) {
+                    if ((c & 63) == 0) stage_acquire();
+                    stage_put32(ebuf, (c >> 5) & 1, o, inv);
+                    if ((c & 63) == 32) stage_flush(to, ebuf, c - 32, g.head, tok_w);
+                } else if (row_ok) {
+                    store_row32(dst + c, o, inv);
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
@@ -770,7 +848,8 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
         if (ok && b->last[X]) {
             __threadfence();
             merge_parts<D>(p, g, X, r, row_ok, keep, tO, m, l, dst,
-                           p.lse ? p.lse + (size_t)tok * p.heads + g.head : nullptr);
+                           p.lse ? p.lse + (size_t)tok * p.heads + g.head : nullptr, to, ebuf,
+                           warp_full, tok_w);
         }
         if (keep) {
             tc_fence_before();
@@ -778,12 +857,16 @@ __device__ void softmax_epilogue(const AttnParams& p, Bars* b, uint32_t tmem, in
             if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->o_empty[X]));
         }
     }
+    // this warp's output stores are complete before the CTA ends
+    if ((threadIdx.x & 31) == 0) bulk_wait_all();
+    __syncwarp();
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams p) {
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                const __grid_constant__ AttnParams p) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -831,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-        softmax_epilogue<D>(p, b, tmem, warp / 4 - 1);
+        softmax_epilogue<D>(p, &to, smem, b, tmem, warp / 4 - 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -844,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const AttnParams& p, cudaStream_t s) {
+                     const CUtensorMap& to, const AttnParams& p, cudaStream_t s) {
     using C = Cfg<D>;
     static bool configured = false;
     if (!configured) {
@@ -853,7 +936,7 @@ cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    attn_kernel<D><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, p);
+    attn_kernel<D><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -877,14 +960,14 @@ cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-static_assert(sizeof(AttnParams) + 3 * sizeof(CUtensorMap) <= 4096,
+static_assert(sizeof(AttnParams) + 4 * sizeof(CUtensorMap) <= 4096,
               "attention kernel parameters beyond 4 KB");
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, cudaStream_t s) {
+                        const CUtensorMap& to, const AttnParams& p, cudaStream_t s) {
     if (p.grid <= 0 || p.total <= 0) return cudaErrorInvalidValue;
-    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, p, s);
-    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, p, s);
+    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, to, p, s);
+    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, to, p, s);
     return cudaErrorInvalidValue;
 }
 

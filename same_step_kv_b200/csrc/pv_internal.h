@@ -18,6 +18,7 @@ using bf16 = __nv_bfloat16;
 constexpr int kMaxSteps = 8;              // denoising steps per chunk a handle may hold
 constexpr int kQRows = 128;               // query rows per tensor-core tile (MMA M)
 constexpr int kQTilesPerCta = 2;          // two query tiles share each K/V tile
+constexpr int kOutRows = 32;               // output rows of one TMA store (one softmax warp)
 constexpr int kQBlock = kQRows * kQTilesPerCta;
 constexpr int kKeyTile = 128;             // keys per K/V tile (MMA N of Q K^T)
 constexpr int kMaxGrid = 160;             // CTAs of one attention launch at most (>= SMs)
@@ -91,7 +92,7 @@ struct AttnParams {
 __host__ __device__ inline size_t partial_slot_floats(int D) { return (size_t)kQRows * D + 2 * kQRows; }
 
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, cudaStream_t s);
+                        const CUtensorMap& to, const AttnParams& p, cudaStream_t s);
 
 // One bounded device wait that runs out (failure-path self-test).
 cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s);
@@ -106,6 +107,8 @@ cudaError_t launch_x0(float* x0, const float* x, const float* v, size_t n, float
 // ----------------------------------------------------------------- host helpers
 // Encodes a 2D bf16 tensor map over `rows` rows of `D` elements with a
 // 64-element x 128-row box and the 128-byte swizzle.
+bool encode_out_map(CUtensorMap* map, void* out, long long tokens, int heads, int D, char* err,
+                    size_t errlen);
 bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, char* err,
                      size_t errlen);
 

@@ -136,12 +136,13 @@ extern "C" pv_status pv_attn_dense_noalloc(const void* q, const void* k, const v
     a.out_tok0 = 0;
     if (plan_attention(p, n_sm, n_part, kMaxCounters) < 0)
         return report_error(PV_ERR_CAPACITY, "pv_attn_dense_noalloc: no plan fits the scratch");
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_rows_map(&tq, q, (long long)heads * n_q, head_dim, msg, sizeof msg) ||
         !encode_rows_map(&tk, k, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
-        !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg))
+        !encode_rows_map(&tv, v, (long long)heads * n_k, head_dim, msg, sizeof msg) ||
+        !encode_out_map(&to, out, n_q, heads, head_dim, msg, sizeof msg))
         return report_error(PV_ERR_CUDA, msg);
-    e = launch_attn(tq, tk, tv, p, st);
+    e = launch_attn(tq, tk, tv, to, p, st);
     if (e != cudaSuccess) {
         snprintf(msg, sizeof msg, "pv_attn_dense_noalloc launch: %s", cudaGetErrorString(e));
         return report_error(PV_ERR_CUDA, msg);
