@@ -25,6 +25,8 @@
 
 namespace pv {
 
+constexpr long long kItemOverhead = 1;  // key-tile equivalents of one segment's fixed work
+
 int plan_attention(AttnParams& p, int n_sm, int part_capacity, int cnt_capacity) {
     long long total = 0;
     int items = 0, max_kt = 0;
@@ -54,19 +56,24 @@ int plan_attention(AttnParams& p, int n_sm, int part_capacity, int cnt_capacity)
         p.item_aligned = 2;  // equal item counts, computed on the device
         return p.grid;
     }
-    // item-aligned: each CTA starts at the item start nearest its stream-K
-    // position, keeping at least one item per CTA
+    // item-aligned: each CTA starts at the item whose start is nearest its
+    // share of the cost, keeping at least one item per CTA.  An item costs
+    // its key tiles plus kItemOverhead: a segment's fixed work (Q load,
+    // first-tile softmax, output) measures at about one key-tile iteration.
     p.item_aligned = 1;
-    std::vector<long long> start;
+    std::vector<long long> start;  // cost before item k
     start.reserve(items + 1);
+    long long cost = 0;
     for (int i = 0; i < p.n_streams; ++i)
-        for (int k = 0; k < p.heads * p.st[i].n_qb; ++k)
-            start.push_back(p.st[i].cost0 + (long long)k * p.st[i].n_kt);
-    start.push_back(total);
+        for (int k = 0; k < p.heads * p.st[i].n_qb; ++k) {
+            start.push_back(cost);
+            cost += p.st[i].n_kt + kItemOverhead;
+        }
+    start.push_back(cost);
     int prev = 0;
     p.first_item[0] = 0;
     for (int c = 1; c < p.grid; ++c) {
-        const long long want = (long long)c * total / p.grid;
+        const long long want = (long long)c * cost / p.grid;
         int k = (int)(std::lower_bound(start.begin(), start.end(), want) - start.begin());
         if (k > 0 && want - start[k - 1] < start[k] - want) --k;
         k = std::max(k, prev + 1);
