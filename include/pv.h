@@ -235,6 +235,19 @@ PV_API pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int
                                 void* out, float* lse, void* ws, size_t ws_bytes,
                                 void* cuda_stream);
 
+/* The work plan that pv_attn_varlen would launch for these lengths on a GPU
+ * with n_sm SMs and a workspace of partial_slots split-KV slots (head_dim
+ * 128), without launching anything: host only.  Items are (sequence, head,
+ * 256-query block), each a run of ceil(n_k / 128) key tiles, laid out
+ * query-block-major and end to end; CTA c processes the key tiles
+ * [ranges[c], ranges[c + 1]) of that list.
+ *  grid: CTAs; ranges: host array of at least min(n_sm, 160) + 1 entries.
+ *  mode: 0 stream-K (equal ranges; split items are merged by the last CTA
+ *  to arrive), 1 item-aligned with cost-balanced starts, 2 item-aligned
+ *  with equal item counts (more than 65,535 items). */
+PV_API pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int heads, int n_sm,
+                              int partial_slots, int* grid, int* mode, long long* ranges);
+
 /* Dense attention like pv_attn_dense (same layouts, same kernel), for
  * callers that cannot allocate device memory where they call it: code inside
  * a custom allocator or memory-pool callback, plugins whose host framework

@@ -849,6 +849,47 @@ pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs
     return PV_OK;
 }
 
+pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int heads, int n_sm,
+                       int partial_slots, int* grid, int* mode, long long* ranges) {
+    if (!grid || !mode || !ranges) return fail(PV_ERR_INVALID_ARG, "NULL output pointer");
+    long long tot_q, tot_k;
+    size_t n_cnt, tiles;
+    pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, 128, &tot_q, &tot_k, &n_cnt, &tiles);
+    if (st) return st;
+    if (tot_q == 0) return fail(PV_ERR_SHAPE, "no queries");
+    if (n_sm < 1 || partial_slots < 0) return fail(PV_ERR_INVALID_ARG, "n_sm < 1 or slots < 0");
+    AttnParams p{};
+    p.heads = heads;
+    int ns = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+        if (n_q[i] == 0) continue;
+        p.st[ns].n_q = n_q[i];
+        p.st[ns].n_k = n_k[i];
+        ++ns;
+    }
+    p.n_streams = ns;
+    if (plan_attention(p, n_sm, partial_slots, (int)n_cnt) < 0)
+        return fail(PV_ERR_CAPACITY, "no plan fits");
+    *grid = p.grid;
+    *mode = p.item_aligned;
+    // the key-tile range of every CTA, as the kernel derives it
+    std::vector<long long> item_start;
+    for (int i = 0; i < p.n_streams; ++i)
+        for (int k = 0; k < heads * p.st[i].n_qb; ++k)
+            item_start.push_back(p.st[i].cost0 + (long long)k * p.st[i].n_kt);
+    item_start.push_back(p.total);
+    for (int c = 0; c <= p.grid; ++c) {
+        if (p.item_aligned == 0) {
+            ranges[c] = (long long)c * p.total / p.grid;
+        } else {
+            const long long k = p.item_aligned == 1 ? (long long)p.first_item[c]
+                                                    : (long long)c * p.n_items / p.grid;
+            ranges[c] = item_start[std::min<long long>(k, p.n_items)];
+        }
+    }
+    return PV_OK;
+}
+
 pv_status pv_euler_step(float* x, const float* v, size_t n, float dsigma, void* cuda_stream) {
     if (n == 0) return PV_OK;
     if (!x || !v) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");

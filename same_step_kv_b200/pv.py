@@ -82,6 +82,8 @@ _SIGS = {
     "pv_kv_selftest_wait_timeout": ([_vp, _vp], _i),
     "pv_attn_varlen_ws_bytes": ([_i, _vp, _vp, _i, _i, ctypes.POINTER(_sz)], _i),
     "pv_attn_varlen": ([_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
+    "pv_attn_plan": ([_i, _vp, _vp, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                      ctypes.POINTER(ctypes.c_longlong)], _i),
     "pv_sigma_schedule": ([_i, ctypes.c_double, ctypes.c_double, ctypes.POINTER(ctypes.c_double),
                            ctypes.POINTER(_i)], _i),
     "pv_euler_cfg_step": ([_vp, _vp, _vp, _sz, ctypes.c_float, ctypes.c_float, _vp], _i),
@@ -236,6 +238,19 @@ def pv_attn_varlen(q, k, v, n_q, n_k, heads, head_dim, out, lse, ws, ws_bytes,
     _check(lib.pv_attn_varlen(_ptr(q), _ptr(k), _ptr(v), len(n_q), _lengths(n_q), _lengths(n_k),
                               heads, head_dim, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
                               _stream(cuda_stream)))
+
+
+def pv_attn_plan(n_q, n_k, heads, n_sm=148, partial_slots=None):
+    """(grid, mode, ranges) of the attention plan for these lengths (host only)."""
+    if len(n_q) != len(n_k):
+        raise ValueError("n_q and n_k differ in length")
+    if partial_slots is None:
+        partial_slots = 4 * 160
+    grid, mode = _i(), _i()
+    ranges = (ctypes.c_longlong * 161)()
+    _check(lib.pv_attn_plan(len(n_q), _lengths(n_q), _lengths(n_k), heads, n_sm, partial_slots,
+                            ctypes.byref(grid), ctypes.byref(mode), ranges))
+    return grid.value, mode.value, list(ranges[:grid.value + 1])
 
 
 def pv_attn_dense_noalloc(q, k, v, n_q, n_k, heads, head_dim, out, lse=None,
