@@ -152,3 +152,38 @@ def test_dense_video_18480(pv):
         o_ref, _ = attention.attend(qr, kr, f64(v[:, hd]))
         assert_attn_close(f64(out[rows, hd]), o_ref, f"dense video head {hd}")
     store.close()
+
+
+def test_dense_score_spikes_force_rescale(pv):
+    """A later key tile whose scores exceed the running maximum by more than 64
+    (log2 units): its exponentials would leave the range the speculative pass
+    allows, so the tile is redone against its exact maximum and O is rescaled.
+    Half the heads get such spikes: keys of 5.0 against queries near 2.0 lift
+    the score by ~112 over the first tile's maximum, ~161 in log2 units, and
+    a key of 10.0 further on lifts it by as much again.  Without the rescale
+    those exponentials overflow to inf.  The spikes sit in tiles that are not
+    the first of their segment (24 heads x 32 key tiles over 148 SMs:
+    stream-K segments of ~5 tiles)."""
+    n_q, n_k, heads, dim = 256, 4096, 24, 128
+    g = torch.Generator().manual_seed(5)
+    q = (2.0 + 0.01 * torch.randn(heads, n_q, dim, generator=g)).to(torch.bfloat16)
+    k = (0.3 * torch.randn(heads, n_k, dim, generator=g)).to(torch.bfloat16)
+    v = torch.randn(heads, n_k, dim, generator=g).to(torch.bfloat16)
+    q[heads // 2:] = torch.randn(heads - heads // 2, n_q, dim, generator=g).to(torch.bfloat16)
+    for pos in (3 * 128 + 5, 9 * 128 + 77, 17 * 128, 25 * 128 + 127, 30 * 128 + 40):
+        k[: heads // 2, pos] = 5.0
+    k[: heads // 2, 31 * 128 + 9] = 10.0
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty(n_q, heads, dim, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(n_q, heads, dtype=torch.float32, device="cuda")
+    wsb = pv.pv_attn_dense_ws_bytes(n_q, n_k, heads, dim)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_attn_dense(q, k, v, n_q, n_k, heads, dim, out, lse, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32)[0]) == 0   # no wait gave up
+    for hd in (0, 5, 11, 12, 23):
+        o_ref, lse_ref = attention.attend(f64(q[hd]), f64(k[hd]), f64(v[hd]))
+        assert_attn_close(f64(out[:, hd]), o_ref, f"spiky head {hd}")
+        assert_lse_close(f64(lse[:, hd]), lse_ref, f"spiky head {hd}")
+    # with spikes the output is (nearly) the value row of the largest one
+    assert torch.allclose(out[:, 0].float(), v[0, 31 * 128 + 9].float().expand(n_q, dim), atol=2e-2)
