@@ -193,26 +193,27 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-// D[tmem] (+)= A[smem] * B[smem]
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t acc) {
+// Warp-wide forms: every lane of the MMA warp runs the issue loop (so the
+// operands are warp-uniform) and elect.sync picks the one lane that issues.
+__device__ __forceinline__ void tc_commit_e(uint32_t bar) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ss_e(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t acc) {
+__device__ __forceinline__ void mma_ts_e(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
         "r"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
@@ -284,9 +285,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // ----------------------------------------------------------------- schedule
 // CTA c owns the key tiles [bound(c), bound(c+1)) of the launch's item list
@@ -428,6 +426,11 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
 template <int D>
 __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t tmem) {
     using C = Cfg<D>;
+    // every lane waits; the vote reconverges the warp before the next issue
+    auto wspin = [&](uint32_t bar, uint32_t par, Bars* bb, int* err) -> bool {
+        const bool r = mbar_spin(bar, par, bb, err);
+        return __all_sync(0xffffffffu, r);
+    };
     constexpr uint32_t idesc_qk = idesc_bf16(kQRows, kKeyTile, false);
     constexpr uint32_t idesc_pv = idesc_bf16(kQRows, D, true);
     const uint32_t sQ = smem_u32(smem + C::kQOff);
@@ -439,7 +442,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tS, sdesc(qa + off, 16, 1024), sdesc(kb + off, 16, 1024), idesc_qk, kk > 0);
+            mma_ss_e(tS, sdesc(qa + off, 16, 1024), sdesc(kb + off, 16, 1024), idesc_qk, kk > 0);
         }
     };
     auto pv = [&](int X, int stage, bool acc) {
@@ -448,7 +451,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
         const uint32_t vb = sKV + stage * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kKeyTile / 16; ++kk)
-            mma_ts(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
+            mma_ts_e(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
                    (acc || kk > 0) ? 1u : 0u);
     };
     int kv = 0, qseg = 0;
@@ -460,8 +463,8 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     // a segment overwrites O, which the previous segment's epilogue must
     // have read out first.
     auto do_pv = [&](int X, int stage, int j) -> bool {
-        if (j == 0 && !mbar_spin(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
-        if (!mbar_spin(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
+        if (j == 0 && !wspin(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
+        if (!wspin(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
         ++pc[X];
         tc_fence_after();
         pv(X, stage, j > 0);
@@ -471,7 +474,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     Seg g;
     while (ok && it.next(p, g)) {
         const bool hasB = g.rows[1] > 0;
-        if (!(ok = mbar_spin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
+        if (!(ok = wspin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
         ++qseg;
         tc_fence_after();
         const int n = g.n;
@@ -481,44 +484,45 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
             const int vs_prev = (kv + 2 * j - 1) % C::kStages;
             const uint32_t vph_prev = ((kv + 2 * j - 1) / C::kStages) & 1;
             if (j > 0) {
-                if (!(ok = mbar_spin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
+                if (!(ok = wspin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
                            do_pv(0, vs_prev, j - 1)))
                     break;
             }
-            if (!(ok = mbar_spin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
+            if (!(ok = wspin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
             tc_fence_after();
             qk(0, ks);
-            tc_commit(smem_u32(&b->s_full[0]));
+            tc_commit_e(smem_u32(&b->s_full[0]));
             if (hasB) {
                 if (j > 0 && !(ok = do_pv(1, vs_prev, j - 1))) break;
                 qk(1, ks);
-                tc_commit(smem_u32(&b->s_full[1]));
+                tc_commit_e(smem_u32(&b->s_full[1]));
             }
             // one release per iteration: K_j and V_(j-1) are no longer read
-            tc_commit(smem_u32(&b->rel[(ev0 + j) & 7]));
+            tc_commit_e(smem_u32(&b->rel[(ev0 + j) & 7]));
         }
         if (!ok) break;
-        tc_commit(smem_u32(&b->q_empty));  // the Q tiles are free once these S products end
+        tc_commit_e(smem_u32(&b->q_empty));  // the Q tiles are free once these S products end
         const int vs = (kv + 2 * n - 1) % C::kStages;
         const uint32_t vph = ((kv + 2 * n - 1) / C::kStages) & 1;
-        if (!(ok = mbar_spin(smem_u32(&b->kv_full[vs]), vph, b, p.err) && do_pv(0, vs, n - 1)))
+        if (!(ok = wspin(smem_u32(&b->kv_full[vs]), vph, b, p.err) && do_pv(0, vs, n - 1)))
             break;
-        tc_commit(smem_u32(&b->o_full[0]));
+        tc_commit_e(smem_u32(&b->o_full[0]));
         ++oc[0];
         if (hasB) {
             if (!(ok = do_pv(1, vs, n - 1))) break;
-            tc_commit(smem_u32(&b->o_full[1]));
+            tc_commit_e(smem_u32(&b->o_full[1]));
             ++oc[1];
         }
-        tc_commit(smem_u32(&b->rel[(ev0 + n) & 7]));  // V of the last iteration
+        tc_commit_e(smem_u32(&b->rel[(ev0 + n) & 7]));  // V of the last iteration
         kv += 2 * n;
         ev0 += n + 1;
     }
     // every MMA issued by this thread has completed once mma_done flips
-    tc_commit(smem_u32(&b->mma_done));
+    tc_commit_e(smem_u32(&b->mma_done));
     const long long t0 = clock64();
     while (!mbar_try(smem_u32(&b->mma_done), 0) && clock64() - t0 < kWaitCycles) {
     }
+    __syncwarp();
 }
 
 #ifndef PV_TRACK_MAX
@@ -903,8 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 0) {
             if (lane_id == 0) producer<D>(&tq, &tk, &tv, p, smem, b);
         } else if (warp == 1) {
-            if (lane_id == 0) mma_issuer<D>(p, smem, b, tmem);
-            __syncwarp();
+            mma_issuer<D>(p, smem, b, tmem);  // the whole warp; one elected lane issues
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
