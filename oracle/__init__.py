@@ -18,7 +18,10 @@ The oracle computes what the pages define, written out plainly:
 * ``euler``     - the flow-matching Euler update, blog chapter 5 ("UniPC")
   and chapter 1 ("From DDPM to Flow Matching");
 * ``session``   - one stream's same-step KV history driven through a whole
-  chunk schedule (model card, "Inference profile").
+  chunk schedule (model card, "Inference profile");
+* ``projection`` - the q, k, v linear layers and the QK-Norm (RMSNorm of q
+  and k), blog chapter 4, end of "3D RoPE: Letting Tokens Know Where They
+  Are".
 
 Every function is pinned by tests under tests/ that do not re-type its
 formula: closed forms, invariants, brute force and the pages' printed numbers.

@@ -350,3 +350,66 @@ def test_cfg_combine_special_cases():
     # linear in w
     a, b = euler.cfg_combine(u, c, 2.0), euler.cfg_combine(u, c, 4.0)
     np.testing.assert_allclose(b - a, 2.0 * (c - u), atol=1e-13)
+
+
+# --------------------------------------------------------- projection + QK-Norm
+from oracle import projection  # noqa: E402
+
+
+def test_linear_index_order():
+    # identity weights return x; zero weights return the bias; one weight
+    # w[i][j] moves input feature j to output feature i (not j to i transposed)
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 6))
+    np.testing.assert_array_equal(projection.linear(x, np.eye(6)), x)
+    b = rng.standard_normal(4)
+    np.testing.assert_array_equal(projection.linear(x, np.zeros((4, 6)), b), np.tile(b, (5, 1)))
+    w = np.zeros((4, 6))
+    w[1, 3] = 2.5
+    y = projection.linear(x, w)
+    np.testing.assert_array_equal(y[:, 1], 2.5 * x[:, 3])
+    assert np.count_nonzero(y[:, [0, 2, 3]]) == 0
+
+
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(8)
+    y = rng.standard_normal((7, 48))
+    g1 = np.ones(48)
+    eps = projection.EPS
+    out = projection.rms_norm(y, g1)
+    ms = np.mean(y * y, axis=1)
+    # mean of the squared output is ms / (ms + eps)
+    np.testing.assert_allclose(np.mean(out * out, axis=1), ms / (ms + eps), rtol=1e-13)
+    # a constant row a gives a / sqrt(a^2 + eps) times the gain
+    g = rng.standard_normal(48)
+    c = projection.rms_norm(np.full((1, 48), -3.0), g)
+    np.testing.assert_allclose(c[0], -3.0 / math.sqrt(9.0 + eps) * g, rtol=1e-14)
+    # without eps the norm is scale invariant (positive scales)
+    np.testing.assert_allclose(projection.rms_norm(5.0 * y, g, 0.0), projection.rms_norm(y, g, 0.0),
+                               rtol=1e-13)
+    # the gain multiplies feature by feature, after the normalisation
+    np.testing.assert_allclose(projection.rms_norm(y, g), out * g, rtol=1e-14)
+
+
+def test_qkv_split_and_norm_only_on_q_and_k():
+    rng = np.random.default_rng(9)
+    heads, d = 2, 8
+    dim = heads * d
+    x = rng.standard_normal((3, dim))
+    w = rng.standard_normal((3 * dim, dim))
+    b = rng.standard_normal(3 * dim)
+    g_q, g_k = rng.standard_normal(dim), rng.standard_normal(dim)
+    q, k, v = projection.qkv(x, w, b, g_q, g_k, heads)
+    assert q.shape == k.shape == v.shape == (3, heads, d)
+    # v is the plain linear layer, feature f at head f // d, dimension f % d
+    yv = x @ w[2 * dim:].T + b[2 * dim:]
+    for f in range(dim):
+        np.testing.assert_allclose(v[:, f // d, f % d], yv[:, f], rtol=1e-13)
+    # q and k rows have unit RMS over all heads once the gain is divided out
+    for t, gg in ((q, g_q), (k, g_k)):
+        z = t.reshape(3, dim) / gg
+        np.testing.assert_allclose(np.mean(z * z, axis=1), 1.0, rtol=1e-4)
+    # scaling a token scales its v, leaves its q and k (nearly) unchanged
+    q2, k2, v2 = projection.qkv(4.0 * x, w, 4.0 * b, g_q, g_k, heads)
+    np.testing.assert_allclose(v2, 4.0 * v, rtol=1e-13)
+    np.testing.assert_allclose(q2, q, rtol=1e-5)
