@@ -175,6 +175,31 @@ PV_API pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int
                          const void* q, const void* k, const void* v, void* q_rot,
                          void* cuda_stream);
 
+/* Workspace bytes of pv_qkv_rope_append for `tokens` tokens (all listed
+ * streams together) of width dim = heads * head_dim. */
+PV_API pv_status pv_qkv_ws_bytes(int tokens, int dim, size_t* ws_bytes);
+
+/* The q, k, v projection with QK-Norm, then what pv_rope_append does
+ * (blog chapter 4, end of "3D RoPE": q and k each pass through their linear
+ * layer and an RMSNorm; v through its linear layer):
+ *   y = x w^T + bias                       (f32 accumulate)
+ *   q = RMSNorm(y[:, 0:dim]) * g_q,  k = RMSNorm(y[:, dim:2 dim]) * g_k,
+ *   v = y[:, 2 dim:3 dim],  RMSNorm(u) = u / sqrt(mean(u^2) + eps),
+ * over the whole vector of a token (all heads), heads split afterwards
+ * (feature f to head f / head_dim); then 3D RoPE of q and k and the append
+ * of k, v into the per-step store exactly as pv_rope_append, q_rot likewise.
+ *  x: bf16 [tokens][dim] (the listed streams' tokens back to back, in list
+ *     order), w: bf16 [3 dim][dim] (W_q, W_k, W_v rows, a linear layer's
+ *     [out][in]), bias: f32 [3 dim], g_q, g_k: f32 [dim], eps > 0.
+ *  ws: device workspace of pv_qkv_ws_bytes, 256-byte aligned (holds y in
+ *     f32 and the per-token sums of squares; no need to clear it).
+ * Two launches: a tcgen05 GEMM whose epilogue adds the bias and sums the
+ * squares, then the RoPE / append kernel, which applies the norm. */
+PV_API pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer,
+                                    int step, const void* x, const void* w, const float* bias,
+                                    const float* g_q, const float* g_k, float eps, void* q_rot,
+                                    void* ws, size_t ws_bytes, void* cuda_stream);
+
 /* Chunk attention of each listed stream at its current chunk, one launch:
  *  o[q] = sum_k softmax_k(q_rot . k_rot / sqrt(D)) v_k over the stream's key
  *  set at (layer, step): FIRST -> its own F0*T keys of step s; PV_STEP_SINK

@@ -195,6 +195,29 @@ bool encode_out_map(CUtensorMap* map, void* out, long long tokens, int heads, in
     return true;
 }
 
+bool encode_2d_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
+                   long long cols, long long rows, int box_cols, int box_rows, char* err,
+                   size_t errlen) {
+    auto enc = get_encode();
+    if (!enc) {
+        snprintf(err, errlen, "cuTensorMapEncodeTiled is not available from the driver");
+        return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elem_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(err, errlen, "cuTensorMapEncodeTiled failed (%d) for %lld x %lld, box %d x %d",
+                 (int)r, rows, cols, box_rows, box_cols);
+        return false;
+    }
+    return true;
+}
+
 }  // namespace pv
 
 struct pv_kv_s {
@@ -525,28 +548,32 @@ pv_status pv_kv_row_offset(pv_kv kv, int layer, int step, int stream, int head, 
     return PV_OK;
 }
 
-pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer, int step,
-                         const void* q, const void* k, const void* v, void* q_rot,
-                         void* cuda_stream) {
-    if (!kv) return fail(PV_ERR_INVALID_ARG, "handle is NULL");
-    if (!kv->device) return fail(PV_ERR_STATE, "bookkeeping-only handle has no device buffers");
+}  // extern "C"
+
+namespace {
+// RoPE / append parameters of the listed streams at (layer, step): the
+// checks and the destinations that pv_rope_append and pv_qkv_rope_append share.
+// Sets *tokens (all streams) and *max_tok.
+pv_status rope_params(pv_kv kv, int n_streams, const int* streams, int layer, int step,
+                      RopeParams* pp, int* tokens, int* max_tok) {
     pv_status st = check_streams(kv, n_streams, streams);
     if (st) return st;
     const pv_kv_config& c = kv->cfg;
     if (layer < 0 || layer >= c.layers) return fail(PV_ERR_INVALID_ARG, "layer %d out of range", layer);
     if (!(step == PV_STEP_SINK || (step >= 0 && step < c.steps)))
         return fail(PV_ERR_INVALID_ARG, "step %d is neither 0..%d nor PV_STEP_SINK", step, c.steps - 1);
-    if (!q || !k || !v || !q_rot) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q_rot, 16))
-        return fail(PV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-    if ((st = check_async("an earlier launch"))) return st;
-
-    std::lock_guard<std::mutex> lock(kv->mu);
-    RopeParams p{};
-    p.q = (const bf16*)q;
-    p.k = (const bf16*)k;
-    p.v = (const bf16*)v;
-    p.q_rot = (bf16*)q_rot;
+    // validate every stream before changing any state
+    for (int i = 0; i < n_streams; ++i) {
+        const StreamState& s = kv->streams[streams[i]];
+        if (step == PV_STEP_SINK) {
+            if (s.phase != PV_PHASE_BOOT)
+                return fail(PV_ERR_STATE, "stream %d: call pv_kv_begin_sink before the sink pass",
+                            streams[i]);
+        } else if (s.phase != PV_PHASE_FIRST && s.phase != PV_PHASE_STEADY) {
+            return fail(PV_ERR_STATE, "stream %d: no denoising step in phase %d", streams[i], s.phase);
+        }
+    }
+    RopeParams& p = *pp;
     p.k_dst = kv->kbase;
     p.v_dst = kv->vbase;
     p.table = (const float2*)(kv->ws + kv->wl.tab_off);
@@ -561,18 +588,7 @@ pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer,
     p.tab_w0 = p.tab_h0 + c.frame_h * c.rope_pairs_h;
     p.dst_head_stride = kv->ltot;
     p.n_streams = n_streams;
-    // validate every stream before changing any state
-    for (int i = 0; i < n_streams; ++i) {
-        const StreamState& s = kv->streams[streams[i]];
-        if (step == PV_STEP_SINK) {
-            if (s.phase != PV_PHASE_BOOT)
-                return fail(PV_ERR_STATE, "stream %d: call pv_kv_begin_sink before the sink pass",
-                            streams[i]);
-        } else if (s.phase != PV_PHASE_FIRST && s.phase != PV_PHASE_STEADY) {
-            return fail(PV_ERR_STATE, "stream %d: no denoising step in phase %d", streams[i], s.phase);
-        }
-    }
-    int tok = 0, max_tok = 0;
+    int tok = 0, mt = 0;
     for (int i = 0; i < n_streams; ++i) {
         StreamState& s = kv->streams[streams[i]];
         pv_kv_state d;
@@ -594,10 +610,102 @@ pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer,
                              (long long)(c.first_frames + s.slot) * kv->T;
         }
         tok += d.n_queries;
-        max_tok = std::max(max_tok, d.n_queries);
+        mt = std::max(mt, d.n_queries);
     }
+    *tokens = tok;
+    *max_tok = mt;
+    return PV_OK;
+}
+
+// Workspace of pv_qkv_rope_append: y f32 [tokens][3 * dim], then the sums of
+// squares f32 [tokens][2], each 256-byte aligned.
+size_t qkv_y_bytes(long long tokens, int dim) { return round_up((size_t)tokens * 3 * dim * 4, 256); }
+}  // namespace
+
+extern "C" {
+
+pv_status pv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer, int step,
+                         const void* q, const void* k, const void* v, void* q_rot,
+                         void* cuda_stream) {
+    if (!kv) return fail(PV_ERR_INVALID_ARG, "handle is NULL");
+    if (!kv->device) return fail(PV_ERR_STATE, "bookkeeping-only handle has no device buffers");
+    if (!q || !k || !v || !q_rot) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(q_rot, 16))
+        return fail(PV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+    pv_status st;
+    if ((st = check_async("an earlier launch"))) return st;
+    std::lock_guard<std::mutex> lock(kv->mu);
+    RopeParams p{};
+    int tok = 0, max_tok = 0;
+    if ((st = rope_params(kv, n_streams, streams, layer, step, &p, &tok, &max_tok))) return st;
+    p.q = (const bf16*)q;
+    p.k = (const bf16*)k;
+    p.v = (const bf16*)v;
+    p.q_rot = (bf16*)q_rot;
     cudaError_t e = launch_rope(p, max_tok, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(e, "rope_append launch");
+    return PV_OK;
+}
+
+pv_status pv_qkv_ws_bytes(int tokens, int dim, size_t* ws_bytes) {
+    if (!ws_bytes) return fail(PV_ERR_INVALID_ARG, "output pointer is NULL");
+    if (tokens < 1 || dim < 64 || dim % 64 != 0)
+        return fail(PV_ERR_SHAPE, "tokens must be positive and dim a multiple of 64");
+    *ws_bytes = qkv_y_bytes(tokens, dim) + round_up((size_t)tokens * 2 * 4, 256);
+    return PV_OK;
+}
+
+pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer, int step,
+                             const void* x, const void* w, const float* bias, const float* g_q,
+                             const float* g_k, float eps, void* q_rot, void* ws, size_t ws_bytes,
+                             void* cuda_stream) {
+    if (!kv) return fail(PV_ERR_INVALID_ARG, "handle is NULL");
+    if (!kv->device) return fail(PV_ERR_STATE, "bookkeeping-only handle has no device buffers");
+    if (!x || !w || !bias || !g_q || !g_k || !q_rot || !ws)
+        return fail(PV_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(q_rot, 16) || !aligned(ws, 256) ||
+        !aligned(bias, 4) || !aligned(g_q, 4) || !aligned(g_k, 4))
+        return fail(PV_ERR_INVALID_ARG, "x, w, q_rot 16-byte, ws 256-byte, vectors 4-byte aligned");
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(PV_ERR_INVALID_ARG, "eps must be > 0");
+    const pv_kv_config& c = kv->cfg;
+    const int dim = c.heads * c.head_dim;
+    if (qkv_gemm_tile_n(dim) == 0)
+        return fail(PV_ERR_SHAPE, "heads * head_dim = %d is not a multiple of 64", dim);
+    pv_status st;
+    if ((st = check_async("an earlier launch"))) return st;
+    std::lock_guard<std::mutex> lock(kv->mu);
+    RopeParams p{};
+    int tok = 0, max_tok = 0;
+    if ((st = rope_params(kv, n_streams, streams, layer, step, &p, &tok, &max_tok))) return st;
+    size_t need = 0;
+    pv_qkv_ws_bytes(tok, dim, &need);
+    if (ws_bytes < need)
+        return fail(PV_ERR_CAPACITY, "workspace of %zu bytes, need %zu", ws_bytes, need);
+    float* y = (float*)ws;
+    float* ss = (float*)((char*)ws + qkv_y_bytes(tok, dim));
+    CUtensorMap tx, tw, ty;
+    char msg[256];
+    const int bn = qkv_gemm_tile_n(dim);
+    if (!encode_2d_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dim, tok, 64, 128, msg,
+                       sizeof msg) ||
+        !encode_2d_map(&tw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dim, 3LL * dim, 64, bn, msg,
+                       sizeof msg) ||
+        !encode_2d_map(&ty, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 3LL * dim, tok, 32, 32, msg,
+                       sizeof msg))
+        return fail(PV_ERR_CUDA, "%s", msg);
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    cudaError_t e = cudaMemsetAsync(ss, 0, (size_t)tok * 2 * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the sums of squares");
+    e = launch_qkv_gemm(tx, tw, ty, bias, ss, tok, dim, (int*)(kv->ws + kv->wl.err_off), s);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv projection launch");
+    p.y = y;
+    p.ss = ss;
+    p.g_q = g_q;
+    p.g_k = g_k;
+    p.eps = eps;
+    p.q_rot = (bf16*)q_rot;
+    e = launch_rope(p, max_tok, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv rope_append launch");
     return PV_OK;
 }
 

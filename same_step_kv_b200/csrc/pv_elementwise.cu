@@ -25,8 +25,13 @@ __device__ __forceinline__ uint32_t pack(float lo, float hi) {
 // "3D RoPE": pair p of a head belongs to the time, height or width block and
 // turns by that coordinate times the pair's frequency, as the complex product
 // (x + i y) e^{i angle}.  One thread handles 8 consecutive dimensions (4
-// pairs, one 16-byte vector) of one (token, head) of q, k and v; rows are
-// read and written with 128-bit coalesced accesses.
+// pairs) of one (token, head) of q, k and v; rows are read and written with
+// 128-bit coalesced accesses.
+// kProj = false: q, k, v are bf16 [tokens][H][D].
+// kProj = true: they are the f32 projection y [tokens][3 * dim] (pv_gemm.cu)
+// and q, k get the rest of the QK-Norm first (same chapter): times
+// rsqrt(ss / dim + eps), ss the token's sum of squares, then the gain.
+template <bool kProj>
 __global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant__ RopeParams p) {
     const RopeStreamDesc& sd = p.st[blockIdx.y];
     const int G = p.head_dim >> 3;                   // 16-byte groups per head row
@@ -38,16 +43,50 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant_
         const int j = it - t * per_tok;
         const int h = j / G;
         const int g = j - h * G;
-        const size_t in_off = ((size_t)(sd.in_tok0 + t) * p.heads + h) * p.head_dim + g * 8;
-        const uint4 qv = ld_stream(p.q + in_off);
-        const uint4 kv = ld_stream(p.k + in_off);
-        const uint4 vv = ld_stream(p.v + in_off);
+        float qf[8], kf[8];
+        uint4 vv;
+        if (kProj) {
+            const int dim = p.heads * p.head_dim;
+            const int f0 = h * p.head_dim + g * 8;           // feature of this group
+            const size_t row = (size_t)(sd.in_tok0 + t);
+            const float* yq = p.y + row * 3 * dim + f0;
+            const float sq = rsqrtf(__ldg(p.ss + row * 2) / dim + p.eps);
+            const float sk = rsqrtf(__ldg(p.ss + row * 2 + 1) / dim + p.eps);
+            const float4 q0 = __ldcs(reinterpret_cast<const float4*>(yq));
+            const float4 q1 = __ldcs(reinterpret_cast<const float4*>(yq + 4));
+            const float4 k0 = __ldcs(reinterpret_cast<const float4*>(yq + dim));
+            const float4 k1 = __ldcs(reinterpret_cast<const float4*>(yq + dim + 4));
+            const float4 v0 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim));
+            const float4 v1 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim + 4));
+            const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                qf[i] = qa[i] * sq * __ldg(p.g_q + f0 + i);
+                kf[i] = ka[i] * sk * __ldg(p.g_k + f0 + i);
+            }
+            vv = make_uint4(pack(v0.x, v0.y), pack(v0.z, v0.w), pack(v1.x, v1.y), pack(v1.z, v1.w));
+        } else {
+            const size_t in_off = ((size_t)(sd.in_tok0 + t) * p.heads + h) * p.head_dim + g * 8;
+            const uint4 qv = ld_stream(p.q + in_off);
+            const uint4 kv = ld_stream(p.k + in_off);
+            vv = ld_stream(p.v + in_off);
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 a = unpack(qw[u]);
+                const float2 b = unpack(kw[u]);
+                qf[2 * u] = a.x;
+                qf[2 * u + 1] = a.y;
+                kf[2 * u] = b.x;
+                kf[2 * u + 1] = b.y;
+            }
+        }
         const int f = sd.frame0 + t / T;
         const int r = t % T;
         const int hh = r / p.frame_w;
         const int ww = r - hh * p.frame_w;
-        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
         uint32_t qo[4], ko[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -61,10 +100,10 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant_
                 idx = p.tab_w0 + ww * p.pairs_w + (pair - p.pairs_t - p.pairs_h);
             }
             const float2 cs = __ldg(p.table + idx);
-            const float2 a = unpack(qw[u]);
-            const float2 b = unpack(kw[u]);
-            qo[u] = pack(fmaf(a.x, cs.x, -a.y * cs.y), fmaf(a.x, cs.y, a.y * cs.x));
-            ko[u] = pack(fmaf(b.x, cs.x, -b.y * cs.y), fmaf(b.x, cs.y, b.y * cs.x));
+            const float ax = qf[2 * u], ay = qf[2 * u + 1];
+            const float bx = kf[2 * u], by = kf[2 * u + 1];
+            qo[u] = pack(fmaf(ax, cs.x, -ay * cs.y), fmaf(ax, cs.y, ay * cs.x));
+            ko[u] = pack(fmaf(bx, cs.x, -by * cs.y), fmaf(bx, cs.y, by * cs.x));
         }
         const size_t qrow = (size_t)sd.qrot_row0 + (size_t)h * sd.n_tok + t;
         st16(p.q_rot + qrow * p.head_dim + g * 8, make_uint4(qo[0], qo[1], qo[2], qo[3]));
@@ -180,7 +219,10 @@ cudaError_t launch_rope(const RopeParams& p, int max_tok, cudaStream_t s) {
     const int per_stream = (int)std::min<long long>((items + 255) / 256,
                                                     std::max(1, 8 * sm_count() / p.n_streams));
     dim3 grid(per_stream, p.n_streams);
-    rope_append_kernel<<<grid, 256, 0, s>>>(p);
+    if (p.y)
+        rope_append_kernel<true><<<grid, 256, 0, s>>>(p);
+    else
+        rope_append_kernel<false><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

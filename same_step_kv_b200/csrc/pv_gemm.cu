@@ -1,0 +1,316 @@
+// The q, k, v projection of the tokens as one tcgen05 GEMM, with the first
+// half of the QK-Norm in its epilogue.
+//
+// y[t][n] = sum_c x[t][c] * w[n][c] + b[n] for the tokens t of a launch and
+// the 3 * dim output features n (q, then k, then v; w stored [out][in] as a
+// linear layer keeps it), kept in f32, and for each token the sums of squares
+// of its q features and of its k features, ss[t][0] and ss[t][1].  The second
+// half of the norm (scale by rsqrt(ss / dim + eps) and the gain) runs where y
+// is read next, in the RoPE / append kernel.  Blog "Learning Video Generation
+// from the Wan2.2 Source Code", chapter 4, end of "3D RoPE": q and k pass
+// through their linear layers, then an RMSNorm.
+//
+// One CTA computes a 128-token x BN-feature tile: warp 0 loads 64-column
+// slices of x and w with TMA into a 4-stage ring (128-byte swizzle), warp 1
+// runs the issue loop with all lanes and one elected lane issues the
+// tcgen05.mma (M = 128, N = BN, K = 16, f32 accumulator in TMEM), warps 4-7
+// (one TMEM lane quadrant each, one token per thread) add the bias, sum the
+// squares and stage the tile in the freed ring for TMA stores.  Every wait on
+// an mbarrier is bounded.
+#include "pv_internal.h"
+
+namespace pv {
+namespace {
+
+constexpr int kGThreads = 256;
+constexpr int kGM = 128;      // tokens per tile
+constexpr int kGK = 64;       // input features per stage (one 128-byte swizzle row of bf16)
+constexpr int kGStages = 4;
+constexpr long long kGWait = 2000000000LL;  // ~1 s of clock64
+
+template <int BN>
+struct GCfg {
+    static constexpr int kABytes = kGM * kGK * 2;
+    static constexpr int kBBytes = BN * kGK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kBarOff = kGStages * kStageBytes;
+    static constexpr int kSmem = kBarOff + 256 + 1024;
+    // the epilogue stages 4 warps x 32 tokens x BN f32 in the freed ring
+    static_assert(4 * 32 * BN * 4 <= kBarOff, "epilogue staging does not fit the ring");
+};
+
+struct GBars {
+    uint64_t full[kGStages];   // the stage's x and w slices have landed
+    uint64_t empty[kGStages];  // the MMAs reading the stage are done
+    uint64_t done;             // every MMA of the tile is done
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t g_smem(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void g_mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void g_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool g_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: false after ~1 s (the error word is set and the CTA aborts)
+// or once another role of the CTA has aborted.
+__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t parity, GBars* b, int* err) {
+    if (g_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!g_try(bar, parity)) {
+        if (*(volatile int*)&b->abort) return false;
+        if (clock64() - t0 > kGWait) {
+            atomicExch(err, 1);
+            *(volatile int*)&b->abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+__device__ __forceinline__ void g_tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                           uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void g_tma_store(const CUtensorMap* map, uint32_t src, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(src)
+        : "memory");
+}
+__device__ __forceinline__ void g_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void g_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// issued by the lane that elect.sync picks; the whole warp executes it
+__device__ __forceinline__ void g_commit(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            bar)
+        : "memory");
+}
+__device__ __forceinline__ void g_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                      uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (version 1)
+__device__ __forceinline__ uint64_t g_desc(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+// kind::f16 instruction descriptor: bf16 A and B (K-major), f32 D, M x N
+__host__ __device__ constexpr uint32_t g_idesc(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void g_tmem_ld32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGThreads, 1)
+    qkv_gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+                    const __grid_constant__ CUtensorMap ty, const float* __restrict__ bias,
+                    float* __restrict__ ss, int tokens, int dim, int* err) {
+    using C = GCfg<BN>;
+    extern __shared__ __align__(1024) uint8_t g_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(g_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    GBars* b = reinterpret_cast<GBars*>(smem + C::kBarOff);
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * kGM;
+    const int n0 = blockIdx.y * BN;
+    const int nk = dim / kGK;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            g_mbar_init(g_smem(&b->full[s]), 1);
+            g_mbar_init(g_smem(&b->empty[s]), 1);
+        }
+        g_mbar_init(g_smem(&b->done), 1);
+        b->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         g_smem(&b->tmem)),
+                     "r"((uint32_t)BN)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    g_fence_before();
+    __syncthreads();
+    g_fence_after();
+    const uint32_t tmem = b->tmem;
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: x rows m0.., w rows n0.., 64 input features per stage
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % kGStages;
+                if (kb >= kGStages &&
+                    !g_wait(g_smem(&b->empty[s]), ((kb / kGStages) - 1) & 1, b, err))
+                    break;
+                const uint32_t full = g_smem(&b->full[s]);
+                g_expect_tx(full, C::kStageBytes);
+                const uint32_t st = g_smem(smem + s * C::kStageBytes);
+                g_tma_load(st, &tx, kb * kGK, m0, full);
+                g_tma_load(st + C::kABytes, &tw, kb * kGK, n0, full);
+                ++issued;
+            }
+            // no copy of ours may still be landing when the CTA leaves
+            for (int i = issued > kGStages ? issued - kGStages : 0; i < issued; ++i) {
+                const long long t0 = clock64();
+                while (!g_try(g_smem(&b->full[i % kGStages]), (i / kGStages) & 1) &&
+                       clock64() - t0 < kGWait) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // MMA issue: the whole warp runs the loop, one elected lane issues
+        constexpr uint32_t idesc = g_idesc(kGM, BN);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % kGStages;
+            if (!__all_sync(0xffffffffu,
+                            g_wait(g_smem(&b->full[s]), (kb / kGStages) & 1, b, err)))
+                break;
+            g_fence_after();
+            const uint32_t a = g_smem(smem + s * C::kStageBytes);
+            const uint32_t bw = a + C::kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kGK / 16; ++kk)
+                g_mma(tmem, g_desc(a + kk * 32), g_desc(bw + kk * 32), idesc,
+                      (kb > 0 || kk > 0) ? 1u : 0u);
+            g_commit(g_smem(&b->empty[s]));  // the stage is free once these MMAs end
+        }
+        g_commit(g_smem(&b->done));
+        // every MMA of ours has ended before TMEM is released
+        const long long t0 = clock64();
+        while (!g_try(g_smem(&b->done), 0) && clock64() - t0 < kGWait) {
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // epilogue: one token per thread, TMEM lane quadrant q4
+        const int q4 = warp - 4;
+        const int grow = m0 + q4 * 32 + lane;
+        const bool ok = __all_sync(0xffffffffu, g_wait(g_smem(&b->done), 0, b, err));
+        if (ok && !*(volatile int*)&b->abort) {
+            g_fence_after();
+            const int kind = n0 / dim;  // 0: q, 1: k, 2: v
+            // 32 tokens x BN f32 of this warp, in 32-column boxes of 4 KB,
+            // staged in the ring that the MMAs no longer read
+            uint8_t* buf = smem + q4 * (32 * BN * 4);
+            float sq = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t o[32];
+                g_tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c, o);
+                uint8_t* box = buf + (c / 32) * 4096;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float* bj = bias + n0 + c + 4 * j;
+                    float4 v;
+                    v.x = __uint_as_float(o[4 * j + 0]) + __ldg(bj + 0);
+                    v.y = __uint_as_float(o[4 * j + 1]) + __ldg(bj + 1);
+                    v.z = __uint_as_float(o[4 * j + 2]) + __ldg(bj + 2);
+                    v.w = __uint_as_float(o[4 * j + 3]) + __ldg(bj + 3);
+                    sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
+                    // 16-byte chunk j of row `lane`, 128-byte swizzle
+                    *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0 && m0 + q4 * 32 < tokens) {
+                for (int c = 0; c < BN; c += 32)
+                    g_tma_store(&ty, g_smem(buf + (c / 32) * 4096), n0 + c, m0 + q4 * 32);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+            }
+            __syncwarp();
+            if (kind < 2 && grow < tokens) atomicAdd(ss + (size_t)grow * 2 + kind, sq);
+        }
+    }
+    g_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        g_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"((uint32_t)BN)
+                     : "memory");
+    }
+}
+
+template <int BN>
+cudaError_t launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                           const float* bias, float* ss, int tokens, int dim, int* err,
+                           cudaStream_t s) {
+    using C = GCfg<BN>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(qkv_gemm_kernel<BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid((tokens + kGM - 1) / kGM, 3 * dim / BN);
+    qkv_gemm_kernel<BN><<<grid, kGThreads, C::kSmem, s>>>(tx, tw, ty, bias, ss, tokens, dim, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int qkv_gemm_tile_n(int dim) {
+    return dim % 256 == 0 ? 256 : dim % 128 == 0 ? 128 : dim % 64 == 0 ? 64 : 0;
+}
+
+cudaError_t launch_qkv_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                            const float* bias, float* ss, int tokens, int dim, int* err,
+                            cudaStream_t s) {
+    switch (qkv_gemm_tile_n(dim)) {
+        case 256: return launch_gemm_bn<256>(tx, tw, ty, bias, ss, tokens, dim, err, s);
+        case 128: return launch_gemm_bn<128>(tx, tw, ty, bias, ss, tokens, dim, err, s);
+        case 64: return launch_gemm_bn<64>(tx, tw, ty, bias, ss, tokens, dim, err, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pv

@@ -45,6 +45,13 @@ struct RopeParams {
     int pairs_t, pairs_h, pairs_w;
     int tab_h0, tab_w0;     // table offsets of the height and width blocks
     long long dst_head_stride;  // destination rows between heads
+    // projection input instead of q, k, v (pv_qkv_rope_append): y f32
+    // [tokens][3 * dim], ss the q / k sums of squares per token, gains g_q, g_k
+    const float* y;
+    const float* ss;
+    const float* g_q;
+    const float* g_k;
+    float eps;
     int n_streams;
     RopeStreamDesc st[PV_MAX_STREAMS];
 };
@@ -98,6 +105,15 @@ cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s);
 
 // ----------------------------------------------------------------- Euler
+// q, k, v projection (pv_gemm.cu): y = x w^T + b in f32 and the q / k sums of
+// squares per token; tiles of 128 tokens x qkv_gemm_tile_n(dim) features.
+int qkv_gemm_tile_n(int dim);
+cudaError_t launch_qkv_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
+                            const float* bias, float* ss, int tokens, int dim, int* err,
+                            cudaStream_t s);
+bool encode_2d_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
+                   long long cols, long long rows, int box_cols, int box_rows, char* err,
+                   size_t errlen);
 cudaError_t launch_euler(float* x, const float* v, size_t n, float dsigma, cudaStream_t s);
 cudaError_t launch_euler_cfg(float* x, const float* vc, const float* vu, size_t n, float w,
                              float dsigma, cudaStream_t s);

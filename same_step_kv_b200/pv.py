@@ -84,6 +84,9 @@ _SIGS = {
     "pv_attn_varlen": ([_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "pv_attn_plan": ([_i, _vp, _vp, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                       ctypes.POINTER(ctypes.c_longlong)], _i),
+    "pv_qkv_ws_bytes": ([_i, _i, ctypes.POINTER(_sz)], _i),
+    "pv_qkv_rope_append": ([_vp, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp,
+                            _vp, _sz, _vp], _i),
     "pv_sigma_schedule": ([_i, ctypes.c_double, ctypes.c_double, ctypes.POINTER(ctypes.c_double),
                            ctypes.POINTER(_i)], _i),
     "pv_euler_cfg_step": ([_vp, _vp, _vp, _sz, ctypes.c_float, ctypes.c_float, _vp], _i),
@@ -238,6 +241,20 @@ def pv_attn_varlen(q, k, v, n_q, n_k, heads, head_dim, out, lse, ws, ws_bytes,
     _check(lib.pv_attn_varlen(_ptr(q), _ptr(k), _ptr(v), len(n_q), _lengths(n_q), _lengths(n_k),
                               heads, head_dim, _ptr(out), _ptr(lse), _ptr(ws), ws_bytes,
                               _stream(cuda_stream)))
+
+
+def pv_qkv_ws_bytes(tokens, dim) -> int:
+    a = _sz()
+    _check(lib.pv_qkv_ws_bytes(tokens, dim, ctypes.byref(a)))
+    return a.value
+
+
+def pv_qkv_rope_append(kv, streams, layer, step, x, w, bias, g_q, g_k, eps, q_rot, ws, ws_bytes,
+                       cuda_stream=None) -> None:
+    n, arr = _streams(streams)
+    _check(lib.pv_qkv_rope_append(kv, n, arr, layer, step, _ptr(x), _ptr(w), _ptr(bias),
+                                  _ptr(g_q), _ptr(g_k), ctypes.c_float(eps), _ptr(q_rot), _ptr(ws),
+                                  ws_bytes, _stream(cuda_stream)))
 
 
 def pv_attn_plan(n_q, n_k, heads, n_sm=148, partial_slots=None):

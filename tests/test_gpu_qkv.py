@@ -1,0 +1,167 @@
+"""q, k, v projection with QK-Norm, RoPE and the append (pv_qkv_rope_append)
+on the GPU against the fp64 oracle (oracle/projection.py, oracle/rope.py):
+q_rot and the K rows within the bf16 RoPE bound, V rows within half a bf16
+ulp plus the f32 accumulation, rows placed where the schedule puts them, for
+the three GEMM tile widths (dim a multiple of 256, 128 and 64 only) and two
+streams in one call."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import assert_rope_close, f64
+from oracle import projection, rope
+from same_step_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+EPS = 1e-6
+
+
+@pytest.fixture(scope="module")
+def pv():
+    from same_step_kv_b200 import pv as m
+    return m
+
+
+def _weights(heads, d, seed):
+    dim = heads * d
+    w = (synth.normal_f32(synth.seed_of(0x0A1, seed), (3 * dim, dim)) / dim ** 0.5).to(torch.bfloat16)
+    b = 0.1 * synth.normal_f32(synth.seed_of(0x0A2, seed), (3 * dim,))
+    g_q = 1.0 + 0.1 * synth.normal_f32(synth.seed_of(0x0A3, seed), (dim,))
+    g_k = 1.0 + 0.1 * synth.normal_f32(synth.seed_of(0x0A4, seed), (dim,))
+    return w.cuda(), b.cuda(), g_q.cuda(), g_k.cuda()
+
+
+def _assert_v_close(got, ref, what):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-5 * np.sqrt(np.mean(ref * ref))
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), f"{what}: {int(bad.sum())} values outside the bound"
+
+
+def _oracle(x, w, b, g_q, g_k, heads, W, Hh, frame0, D, rows=None):
+    x64 = f64(x) if rows is None else f64(x)[rows]
+    q, k, v = projection.qkv(x64, f64(w), f64(b), f64(g_q), f64(g_k), heads, EPS)
+    n = x.shape[0]
+    f, hh, ww = rope.token_coords(n, W, Hh, frame0)
+    if rows is not None:
+        f, hh, ww = f[rows], hh[rows], ww[rows]
+    pairs = rope.axis_pairs(D)
+    return rope.rotate(q, f, hh, ww, pairs=pairs), rope.rotate(k, f, hh, ww, pairs=pairs), v
+
+
+@pytest.mark.parametrize("heads,d", [(2, 64), (2, 128), (3, 64)])
+def test_first_chunk_tiny(pv, heads, d):
+    # dim 128, 256 and 192: GEMM tiles of 128, 256 and 64 features
+    W, Hh, R = 8, 4, 2
+    T = W * Hh
+    cfg = pv.make_config(2, heads, d, W, Hh, ring_slots=R, max_streams=2, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    Kr, Vr = st.k_region(), st.v_region()
+    n, layer, step, stream = 3 * T, 1, 2, 1
+    pv.pv_kv_begin_chunk(h, stream, 3)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B1, heads, d), (n, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, heads * 1000 + d)
+    q_rot = torch.empty(heads * n * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(n, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [stream], layer, step, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    qr, kr, v = _oracle(x, w, b, g_q, g_k, heads, W, Hh, 0, d)
+    assert_rope_close(f64(q_rot.view(heads, n, d)), qr.transpose(1, 0, 2), "q_rot")
+    assert_rope_close(f64(Kr[layer, step, stream, :, :n]), kr.transpose(1, 0, 2), "K rows")
+    _assert_v_close(f64(Vr[layer, step, stream, :, :n]), v.transpose(1, 0, 2), "V rows")
+    # nothing else of the store was written (it starts zeroed)
+    assert int(torch.count_nonzero(Kr[layer, step, stream, :, n:])) == 0
+    assert int(torch.count_nonzero(Kr[layer, step, 0])) == 0
+    st.close()
+
+
+def test_steady_chunk_profile(pv):
+    # the profile's steady chunk: 880 tokens of dim 3072 (24 x 128) into ring slot 9
+    W, Hh, heads, d, R = 40, 22, 24, 128, 18
+    T = W * Hh
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    s = pv.pv_kv_state()
+    s.phase, s.chunk = pv.PV_PHASE_STEADY, 28
+    pv.pv_kv_set_state(h, 0, s)
+    s = pv.pv_kv_get_state(h, 0)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B2, 0), (T, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 7)
+    q_rot = torch.empty(heads * T * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(T, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [0], 0, 2, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    rows = np.array([0, 1, 127, 128, 255, 256, 500, 767, 768, 879])
+    qr, kr, v = _oracle(x, w, b, g_q, g_k, heads, W, Hh, s.frame0, d, rows)
+    r0 = 3 * T + s.slot * T
+    Kr, Vr = st.k_region(), st.v_region()
+    assert_rope_close(f64(q_rot.view(heads, T, d)[:, rows]), qr.transpose(1, 0, 2), "q_rot")
+    assert_rope_close(f64(Kr[0, 2, 0, :, r0 + rows]), kr.transpose(1, 0, 2), "K rows")
+    _assert_v_close(f64(Vr[0, 2, 0, :, r0 + rows]), v.transpose(1, 0, 2), "V rows")
+    st.close()
+
+
+def test_two_streams_one_call(pv):
+    # a stream in its first chunk (96 tokens) and one at a steady chunk (32)
+    W, Hh, heads, d, R = 8, 4, 2, 128, 2
+    T = W * Hh
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_streams=2, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    s = pv.pv_kv_state()
+    s.phase, s.chunk = pv.PV_PHASE_STEADY, 5
+    pv.pv_kv_set_state(h, 1, s)
+    s = pv.pv_kv_get_state(h, 1)
+    dim = heads * d
+    n0, n1 = 3 * T, T
+    x = synth.normal_bf16(synth.seed_of(0x0B3, 0), (n0 + n1, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 11)
+    q_rot = torch.empty(heads * (n0 + n1) * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(n0 + n1, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [0, 1], 0, 1, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    Kr, Vr = st.k_region(), st.v_region()
+    # stream 0: tokens 0..95 at frames 0..2, sink rows of step 1
+    qr, kr, v = _oracle(x[:n0], w, b, g_q, g_k, heads, W, Hh, 0, d)
+    assert_rope_close(f64(q_rot[: heads * n0 * d].view(heads, n0, d)), qr.transpose(1, 0, 2), "q0")
+    assert_rope_close(f64(Kr[0, 1, 0, :, :n0]), kr.transpose(1, 0, 2), "K0")
+    # stream 1: tokens 96..127 at its chunk's frame, in its ring slot
+    qr, kr, v = _oracle(x[n0:], w, b, g_q, g_k, heads, W, Hh, s.frame0, d)
+    q1 = q_rot[heads * n0 * d:].view(heads, n1, d)
+    assert_rope_close(f64(q1), qr.transpose(1, 0, 2), "q1")
+    r0 = 3 * T + s.slot * T
+    assert_rope_close(f64(Kr[0, 1, 1, :, r0:r0 + n1]), kr.transpose(1, 0, 2), "K1")
+    _assert_v_close(f64(Vr[0, 1, 1, :, r0:r0 + n1]), v.transpose(1, 0, 2), "V1")
+    st.close()
+
+
+def test_qkv_rejects_bad_arguments(pv):
+    cfg = pv.make_config(1, 2, 64, 8, 4, ring_slots=2, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    x = torch.zeros(96, 128, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(384, 128, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(384, device="cuda")
+    q_rot = torch.empty(2 * 96 * 64, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(96, 128)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pv.PVError) as e:
+        pv.pv_qkv_rope_append(h, [0], 0, 0, x, w, f, f, f, 1e-6, q_rot, ws, wsb - 256)
+    assert e.value.status == pv.PV_ERR_CAPACITY
+    with pytest.raises(pv.PVError):
+        pv.pv_qkv_rope_append(h, [0], 0, 0, x, w, f, f, f, 0.0, q_rot, ws, wsb)
+    with pytest.raises(pv.PVError):
+        pv.pv_qkv_rope_append(h, [0], 0, 0, x, 0, f, f, f, 1e-6, q_rot, ws, wsb)
+    st.close()
