@@ -11,7 +11,7 @@ every layer is pre-filled, and the working set (6.9 GB of K/V) is far larger
 than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload step|cross_attn|sampler]
+                    [--workload step|cross_attn|sampler|qkv]
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 on the host cores on a bounded sample of the same workload.
@@ -308,6 +308,96 @@ def run_cross_attn(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_qkv(args, rank, world, local):
+    """The q, k, v projection with QK-Norm, RoPE and append of the steady chunk
+    (880 tokens of dim 3072 = 24 x 128), one pv_qkv_rope_append per layer
+    (its own weights), 30 layers per step.  Metric: the GEMM's algorithmic
+    FLOPs (2 x 880 x 3072 x 9216 per layer) over the time of the whole call
+    (GEMM + norm / RoPE / append launches)."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    NL = args.layers
+    dim = HEADS * D
+    cfg = pv.make_config(NL, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
+    store = pv.KVStore(cfg, device=dev)
+    h = store.handle
+    st = pv.pv_kv_state()
+    st.phase, st.chunk = pv.PV_PHASE_STEADY, CHUNK
+    pv.pv_kv_set_state(h, 0, st)
+    x = [synth.normal_bf16(synth.seed_of(0x6101, rank, l), (T, dim), dev) for l in range(NL)]
+    w = [(synth.normal_f32(synth.seed_of(0x6102, rank, l), (3 * dim, dim), dev) / dim ** 0.5)
+         .to(torch.bfloat16) for l in range(NL)]
+    bias = [0.1 * synth.normal_f32(synth.seed_of(0x6103, rank, l), (3 * dim,), dev) for l in range(NL)]
+    g = 1.0 + 0.1 * synth.normal_f32(synth.seed_of(0x6104, rank), (2, dim), dev)
+    q_rot = torch.empty(HEADS * T * D, dtype=torch.bfloat16, device=dev)
+    wsb = pv.pv_qkv_ws_bytes(T, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    ev = []
+
+    def call(l, xl):
+        pv.pv_qkv_rope_append(h, [0], l, STEP, xl, w[l], bias[l], g[0], g[1], 1e-6, q_rot, ws, wsb,
+                              cs)
+
+    def step(record):
+        for l in range(NL):
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+            call(l, x[l])
+            if record:
+                e1.record(cs)
+                ev.append((e0, e1))
+
+    ms_step, clocks = timed_steps(step, args, local, world, cs)
+    call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = 2 * T * dim * 3 * dim
+    # e2e: each layer's tokens from pinned host memory, q_rot read back
+    hx = [t.cpu().pin_memory() for t in x]
+    hq = torch.empty(q_rot.shape, dtype=q_rot.dtype).pin_memory()
+    dx = torch.empty_like(x[0])
+
+    def e2e_step(record):
+        for l in range(NL):
+            dx.copy_(hx[l], non_blocking=True)
+            call(l, dx)
+        hq.copy_(q_rot, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        a = flops / (call_ms * 1e-3) / 1e12
+        line = {
+            "metric": "qkv projection TFLOP/s (QK-Norm, RoPE, append fused around a tcgen05 GEMM)",
+            "value": NL * flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"qkv projection of the steady chunk, 880 tokens x {dim} -> "
+                                   f"3 x {dim}, {NL} layers (random weights)",
+                       "l2": f"weights larger than L2 ({NL * 3 * dim * dim * 2 / 1e9:.2f} GB "
+                             "per step), no flush"},
+            "roofline": {"bound": "tensor", "achieved": a, "peak": peak, "unit": "TFLOP/s",
+                         "frac": a / peak, "peak_source": f"{src} bf16_tflops_sustained",
+                         "kernel": "qkv_gemm_kernel<256> + rope_append_kernel<true> (one call)",
+                         "ms_per_launch": call_ms, "traffic": None},
+            "e2e": {"value": NL * flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": NL * T * dim * 2,
+                    "d2h_bytes_per_step": HEADS * T * D * 2},
+            "gpu_launches": 2 * NL * args.steps, "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    store.close()
+
+
 SAMPLER_FRAMES = 248   # 8 streams x 31 latent frames
 
 
@@ -393,12 +483,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers per step (30 in the profile; fewer only for small ncu captures)")
-    ap.add_argument("--workload", default="step", choices=["step", "cross_attn", "sampler"],
-                    help="step: the same-step KV chunk step (default); cross_attn, sampler: "
-                         "the cross-attention and sampler-variant kernels on their own")
+    ap.add_argument("--workload", default="step",
+                    choices=["step", "cross_attn", "sampler", "qkv"],
+                    help="step: the same-step KV chunk step (default); cross_attn, sampler, "
+                         "qkv: the cross-attention, sampler-variant and q/k/v projection "
+                         "kernels on their own")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"step": 100, "cross_attn": 400, "sampler": 2000}[args.workload]
+        args.steps = {"step": 100, "cross_attn": 400, "sampler": 2000, "qkv": 50}[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -409,7 +501,8 @@ def main():
         run_reference(args, rank)
         return
     if args.workload != "step":
-        (run_cross_attn if args.workload == "cross_attn" else run_sampler)(args, rank, world, local)
+        {"cross_attn": run_cross_attn, "sampler": run_sampler, "qkv": run_qkv}[args.workload](
+            args, rank, world, local)
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
