@@ -226,3 +226,22 @@ def test_varlen_workspace_and_shape_checks():
         assert e.value.status == pv.PV_ERR_SHAPE
     # no queries anywhere: a no-op that touches no device
     pv.pv_attn_varlen(0, 0, 0, [0, 0], [3, 0], 2, 64, 0, None, 0, 0)
+
+
+# ------------------------------------------------------------------ q/k/v projection (host checks)
+def test_qkv_workspace_and_host_checks():
+    # y in f32 for 3 * dim features per token, then two sums of squares per token
+    ws = pv.pv_qkv_ws_bytes(880, 3072)
+    y = 880 * 3 * 3072 * 4
+    assert ws == ((y + 255) // 256) * 256 + ((880 * 8 + 255) // 256) * 256
+    for args in ((0, 3072), (880, 100), (880, 0)):
+        with pytest.raises(pv.PVError) as e:
+            pv.pv_qkv_ws_bytes(*args)
+        assert e.value.status == pv.PV_ERR_SHAPE
+    # a bookkeeping-only handle has no store to append into
+    h = pv.pv_kv_init(_cfg(2))
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    with pytest.raises(pv.PVError) as e:
+        pv.pv_qkv_rope_append(h, [0], 0, 0, 16, 16, 16, 16, 16, 1e-6, 16, 256, 1 << 20)
+    assert e.value.status == pv.PV_ERR_STATE
+    pv.pv_kv_destroy(h)
