@@ -11,9 +11,9 @@
 // One CTA = 3 warpgroups (12 warps):
 //   warp 0       TMA producer: the two Q tiles once, then K_j, V_j per key
 //                tile into a ring of shared-memory stages (128-byte swizzle).
-//   warp 1       allocates 512 TMEM columns; one lane issues every
-//                tcgen05.mma: S_X = Q_X K_j^T (SS form), O_X += P_X V_j (P
-//                from TMEM).
+//   warp 1       allocates 512 TMEM columns and runs the MMA issue loop
+//                with all lanes; one elected lane issues each tcgen05.mma:
+//                S_X = Q_X K_j^T (SS form), O_X += P_X V_j (P from TMEM).
 //   warps 2, 3   idle.  Warpgroup 0 gives registers to the other two.
 //   warps 4..7   softmax of query tile A (TMEM lane = query row),
 //   warps 8..11  softmax of query tile B.
@@ -21,6 +21,8 @@
 // P_X (bf16 pairs) overwrites the first 64 columns of S_X.
 // The MMA order PV_A(j-1), S_A(j), PV_B(j-1), S_B(j) lets tile B's softmax run
 // while tile A's products are on the tensor pipe, and the other way round.
+// Each P V is issued in two halves of 64 keys: the softmax hands over the
+// first half of P as soon as it is stored and computes the second meanwhile.
 // The running maximum is only moved when it grows by more than 8 (log2
 // units), so O is rescaled rarely; P stays below 2^8 and the final
 // normalisation uses the m that was actually applied, so the result is exact
@@ -63,6 +65,7 @@ struct Bars {  // 264 bytes, inside the 512 reserved after the tiles
     uint64_t ep_out[2];   // split epilogue: the arrival count is in last[]
     uint64_t s_full[2];
     uint64_t p_full[2];
+    uint64_t p_lo[2];     // [X]: the first 64 key columns of P are in TMEM
     uint64_t o_full[2];
     uint64_t mma_done;
     uint64_t kv_full[8];
@@ -445,12 +448,12 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
             mma_ss_e(tS, sdesc(qa + off, 16, 1024), sdesc(kb + off, 16, 1024), idesc_qk, kk > 0);
         }
     };
-    auto pv = [&](int X, int stage, bool acc) {
+    auto pv = [&](int X, int stage, bool acc, int k0) {
         const uint32_t tS = tmem + X * 128;
         const uint32_t tO = tmem + C::kColsO + X * D;
         const uint32_t vb = sKV + stage * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kKeyTile / 16; ++kk)
+        for (int kk = k0; kk < k0 + kKeyTile / 32; ++kk)
             mma_ts_e(tO, tS + kk * 8, sdesc(vb + kk * 2048, 16384, 1024), idesc_pv,
                    (acc || kk > 0) ? 1u : 0u);
     };
@@ -464,10 +467,13 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     // have read out first.
     auto do_pv = [&](int X, int stage, int j) -> bool {
         if (j == 0 && !wspin(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
+        if (!wspin(smem_u32(&b->p_lo[X]), pc[X] & 1, b, p.err)) return false;
+        tc_fence_after();
+        pv(X, stage, j > 0, 0);          // keys 0..63 while the softmax does 64..127
         if (!wspin(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
         ++pc[X];
         tc_fence_after();
-        pv(X, stage, j > 0);
+        pv(X, stage, true, kKeyTile / 32);
         return true;
     };
     SegIter it(p);
@@ -528,36 +534,29 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
 #ifndef PV_TRACK_MAX
 #define PV_TRACK_MAX 0
 #endif
-// One pass of exponentials over this thread's 128 scores: p = 2^(s*sl2 - m)
-// on the XU pipe, written to TMEM as bf16 pairs over the first 64 columns of
-// S in two 32-column stores (fewer, larger stores than 16-column ones:
-// -3.6 % per launch, measured).  The bf16 value is the upper half of the f32
-// (round toward zero, a byte permute on the ALU pipe instead of a conversion
-// on the XU pipe), and the row sum accumulates exactly those rounded values,
-// so that P and its normaliser agree.
-__device__ __forceinline__ void exp_pass(const uint32_t* sr, float sl2, float m, uint32_t tS,
-                                         float& l_tile) {
-    const float2 sl2x2 = make_float2(sl2, sl2);
-    const float2 nmx2 = make_float2(-m, -m);
+// Exponentials of 64 of this thread's scores: p = 2^(s*sl2 - m) on the XU
+// pipe, written to TMEM as bf16 pairs at tP (32 columns, one store; fewer,
+// larger stores than 16-column ones measured 4 % faster per launch).  The
+// bf16 value is the upper half of the f32 (round toward zero, a byte permute
+// on the ALU pipe instead of a conversion on the XU pipe); the returned sum
+// adds exactly those rounded values, so that P and its normaliser agree.
+__device__ __forceinline__ float exp_half(const uint32_t* sr, float2 sl2x2, float2 nmx2,
+                                          uint32_t tP) {
     float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+    uint32_t pk[32];
 #pragma unroll
-    for (int c0 = 0; c0 < 128; c0 += 64) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-            const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(sr[c0 + i]), __uint_as_float(sr[c0 + i + 1])), sl2x2,
-                nmx2);
-            const uint32_t b0 = __float_as_uint(ex2(x.x)) & 0xFFFF0000u;
-            const uint32_t b1 = __float_as_uint(ex2(x.y)) & 0xFFFF0000u;
-            acc[(i >> 1) & 3] = __fadd2_rn(acc[(i >> 1) & 3],
-                                           make_float2(__uint_as_float(b0), __uint_as_float(b1)));
-            pk[i / 2] = __byte_perm(b0, b1, 0x7632);
-        }
-        tmem_st32(tS + c0 / 2, pk);
+    for (int i = 0; i < 64; i += 2) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                    sl2x2, nmx2);
+        const uint32_t b0 = __float_as_uint(ex2(x.x)) & 0xFFFF0000u;
+        const uint32_t b1 = __float_as_uint(ex2(x.y)) & 0xFFFF0000u;
+        acc[(i >> 1) & 3] =
+            __fadd2_rn(acc[(i >> 1) & 3], make_float2(__uint_as_float(b0), __uint_as_float(b1)));
+        pk[i / 2] = __byte_perm(b0, b1, 0x7632);
     }
+    tmem_st32(tP, pk);
     const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-    l_tile = a.x + a.y;
+    return a.x + a.y;
 }
 
 // Row maximum of 128 scores (masked ones are -inf).
@@ -725,7 +724,6 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
         const AttnStreamDesc& s = p.st[g.si];
         float m = -INFINITY;  // maximum applied to the exponentials, log2 units
         float l = 0.f;        // sum of the exponentials (as rounded into P)
-        float l_tile = 0.f;
         for (int j = 0; j < g.n; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->s_full[X]), sc & 1, b, p.err));
             if (!ok) break;
@@ -739,19 +737,17 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
                 for (int c = 0; c < 128; ++c)
                     if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
             }
-            if (j == 0) m = row_max(sr) * sl2;  // the running maximum starts here
-            // Exponentials with the maximum in hand (it is not recomputed per
-            // tile).  P and the sums stay finite while no score exceeds m by
-            // 64 or more (log2 units): then p < 2^64 and l < 2^71.  If the
-            // tile's sum leaves that range, the tile is redone against its
-            // exact maximum and O is rescaled, as in the plain online softmax.
-            exp_pass(sr, sl2, m, tS, l_tile);
-            if (__any_sync(0xffffffffu, !(l_tile < 1.8446744e19f))) {
-                const float m_new = fmaxf(m, row_max(sr) * sl2);
-                const float alpha = ex2(m - m_new);
-                l *= alpha;
-                m = m_new;
-                if (j > 0) {
+            {
+                // the tile's row maximum; O is rescaled only when it grows by
+                // more than 8 (log2 units), so p stays <= 2^8
+                const float m_t = row_max(sr) * sl2;
+                if (j == 0) {
+                    m = m_t;
+                } else if (__any_sync(0xffffffffu, m_t > m + 8.0f)) {
+                    const float m_new = fmaxf(m, m_t);
+                    const float alpha = ex2(m - m_new);
+                    l *= alpha;
+                    m = m_new;
                     // O holds P V of tiles < j, complete: S(j) was committed after it
 #pragma unroll 1
                     for (int c = 0; c < D; c += 32) {
@@ -763,9 +759,17 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
                         tmem_st32(tO + c, o);
                     }
                 }
-                exp_pass(sr, sl2, m, tS, l_tile);
             }
-            l += l_tile;
+            // P in two halves: the first goes to the tensor pipe (P V of keys
+            // 0..63) while the second half's exponentials are computed
+            const float2 sl2x2 = make_float2(sl2, sl2);
+            const float2 nmx2 = make_float2(-m, -m);
+            l += exp_half(sr, sl2x2, nmx2, tS);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->p_lo[X]));
+            l += exp_half(sr + 64, sl2x2, nmx2, tS + 32);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -878,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&b->s_full[x]), 1);
             mbar_init(smem_u32(&b->p_full[x]), 4);   // one arrive per softmax warp
+            mbar_init(smem_u32(&b->p_lo[x]), 4);
             mbar_init(smem_u32(&b->o_full[x]), 1);
             mbar_init(smem_u32(&b->o_empty[x]), 4);  // one arrive per softmax warp
             mbar_init(smem_u32(&b->ep_in[x]), 4);

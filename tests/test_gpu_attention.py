@@ -155,10 +155,9 @@ def test_dense_video_18480(pv):
 
 
 def test_dense_score_spikes_force_rescale(pv):
-    """A later key tile whose scores exceed the running maximum by more than 64
-    (log2 units): its exponentials would leave the range the speculative pass
-    allows, so the tile is redone against its exact maximum and O is rescaled.
-    Half the heads get such spikes: keys of 5.0 against queries near 2.0 lift
+    """A later key tile whose scores exceed the running maximum by far more
+    than the lazy-rescale threshold (log2 units): the running maximum moves
+    and O and l are rescaled inside a segment.  Half the heads get such spikes: keys of 5.0 against queries near 2.0 lift
     the score by ~112 over the first tile's maximum, ~161 in log2 units, and
     a key of 10.0 further on lifts it by as much again.  Without the rescale
     those exponentials overflow to inf.  The spikes sit in tiles that are not
