@@ -10,38 +10,44 @@
 // from the Wan2.2 Source Code", chapter 4, end of "3D RoPE": q and k pass
 // through their linear layers, then an RMSNorm.
 //
-// One CTA computes a 128-token x BN-feature tile: warp 0 loads 64-column
-// slices of x and w with TMA into a 4-stage ring (128-byte swizzle), warp 1
-// runs the issue loop with all lanes and one elected lane issues the
-// tcgen05.mma (M = 128, N = BN, K = 16, f32 accumulator in TMEM), warps 4-7
-// (one TMEM lane quadrant each, one token per thread) add the bias, sum the
-// squares and stage the tile in the freed ring for TMA stores.  Every wait on
-// an mbarrier is bounded.
+// One CTA computes a 256-token x BN-feature tile as two 128-token halves that
+// share each slice of w in shared memory (half the w traffic per FLOP of a
+// 128-token tile; for the 880 x 3072 chunk the 4 x 36 tiles are one wave on
+// 148 SMs).  Warp 0 loads 64-column slices of x and w with TMA into a ring
+// of stages (128-byte swizzle); warp 1 runs the issue loop with all lanes and
+// one elected lane issues the tcgen05.mma (M = 128, N = BN, K = 16, one f32
+// accumulator per half in TMEM); warps 4-7 (one TMEM lane quadrant each, one
+// token of each half per thread) add the bias, sum the squares and stage the
+// tile in the freed ring for TMA stores.  A half beyond the last token is
+// neither loaded nor multiplied.  Every wait on an mbarrier is bounded.
 #include "pv_internal.h"
 
 namespace pv {
 namespace {
 
 constexpr int kGThreads = 256;
-constexpr int kGM = 128;      // tokens per tile
+constexpr int kGM = 128;      // tokens per half tile (one MMA's M)
+constexpr int kGHalves = 2;   // halves per tile
 constexpr int kGK = 64;       // input features per stage (one 128-byte swizzle row of bf16)
-constexpr int kGStages = 4;
+constexpr int kGMaxStages = 4;
 constexpr long long kGWait = 2000000000LL;  // ~1 s of clock64
 
 template <int BN>
 struct GCfg {
-    static constexpr int kABytes = kGM * kGK * 2;
+    static constexpr int kABytes = kGM * kGK * 2;          // one half's x slice
     static constexpr int kBBytes = BN * kGK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kBarOff = kGStages * kStageBytes;
+    static constexpr int kStageBytes = kGHalves * kABytes + kBBytes;
+    static constexpr int kStages = BN == 256 ? 3 : kGMaxStages;
+    static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr int kSmem = kBarOff + 256 + 1024;
-    // the epilogue stages 4 warps x 32 tokens x BN f32 in the freed ring
+    // the epilogue stages 4 warps x 32 tokens x BN f32 (one half) in the freed ring
     static_assert(4 * 32 * BN * 4 <= kBarOff, "epilogue staging does not fit the ring");
+    static_assert(kBarOff + 256 + 1024 <= 227 * 1024, "shared memory");
 };
 
 struct GBars {
-    uint64_t full[kGStages];   // the stage's x and w slices have landed
-    uint64_t empty[kGStages];  // the MMAs reading the stage are done
+    uint64_t full[kGMaxStages];   // the stage's x and w slices have landed
+    uint64_t empty[kGMaxStages];  // the MMAs reading the stage are done
     uint64_t done;             // every MMA of the tile is done
     uint32_t tmem;
     int abort;
@@ -156,11 +162,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
     GBars* b = reinterpret_cast<GBars*>(smem + C::kBarOff);
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kGM;
+    constexpr int kStages = C::kStages;
+    const int m0 = blockIdx.x * (kGM * kGHalves);
     const int n0 = blockIdx.y * BN;
     const int nk = dim / kGK;
+    const int halves = m0 + kGM < tokens ? 2 : 1;  // the second half holds tokens
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             g_mbar_init(g_smem(&b->full[s]), 1);
             g_mbar_init(g_smem(&b->empty[s]), 1);
         }
@@ -172,7 +180,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          g_smem(&b->tmem)),
-                     "r"((uint32_t)BN)
+                     "r"((uint32_t)(kGHalves * BN))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -182,24 +190,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t tmem = b->tmem;
     if (warp == 0) {
         if (lane == 0) {
-            // producer: x rows m0.., w rows n0.., 64 input features per stage
+            // producer: x rows m0.. (one or two halves), w rows n0.., 64 input
+            // features per stage
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kGStages;
-                if (kb >= kGStages &&
-                    !g_wait(g_smem(&b->empty[s]), ((kb / kGStages) - 1) & 1, b, err))
+                const int s = kb % kStages;
+                if (kb >= kStages && !g_wait(g_smem(&b->empty[s]), ((kb / kStages) - 1) & 1, b, err))
                     break;
                 const uint32_t full = g_smem(&b->full[s]);
-                g_expect_tx(full, C::kStageBytes);
+                g_expect_tx(full, halves * C::kABytes + C::kBBytes);
                 const uint32_t st = g_smem(smem + s * C::kStageBytes);
-                g_tma_load(st, &tx, kb * kGK, m0, full);
-                g_tma_load(st + C::kABytes, &tw, kb * kGK, n0, full);
+                for (int u = 0; u < halves; ++u)
+                    g_tma_load(st + u * C::kABytes, &tx, kb * kGK, m0 + u * kGM, full);
+                g_tma_load(st + kGHalves * C::kABytes, &tw, kb * kGK, n0, full);
                 ++issued;
             }
             // no copy of ours may still be landing when the CTA leaves
-            for (int i = issued > kGStages ? issued - kGStages : 0; i < issued; ++i) {
+            for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i) {
                 const long long t0 = clock64();
-                while (!g_try(g_smem(&b->full[i % kGStages]), (i / kGStages) & 1) &&
+                while (!g_try(g_smem(&b->full[i % kStages]), (i / kStages) & 1) &&
                        clock64() - t0 < kGWait) {
                 }
             }
@@ -208,17 +217,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // MMA issue: the whole warp runs the loop, one elected lane issues
         constexpr uint32_t idesc = g_idesc(kGM, BN);
         for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % kGStages;
+            const int s = kb % kStages;
             if (!__all_sync(0xffffffffu,
-                            g_wait(g_smem(&b->full[s]), (kb / kGStages) & 1, b, err)))
+                            g_wait(g_smem(&b->full[s]), (kb / kStages) & 1, b, err)))
                 break;
             g_fence_after();
             const uint32_t a = g_smem(smem + s * C::kStageBytes);
-            const uint32_t bw = a + C::kABytes;
+            const uint32_t bw = a + kGHalves * C::kABytes;
+            for (int u = 0; u < halves; ++u) {
 #pragma unroll
-            for (int kk = 0; kk < kGK / 16; ++kk)
-                g_mma(tmem, g_desc(a + kk * 32), g_desc(bw + kk * 32), idesc,
-                      (kb > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kGK / 16; ++kk)
+                    g_mma(tmem + u * BN, g_desc(a + u * C::kABytes + kk * 32), g_desc(bw + kk * 32),
+                          idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
             g_commit(g_smem(&b->empty[s]));  // the stage is free once these MMAs end
         }
         g_commit(g_smem(&b->done));
@@ -228,9 +239,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // epilogue: one token per thread, TMEM lane quadrant q4
+        // epilogue: one token of each half per thread, TMEM lane quadrant q4
         const int q4 = warp - 4;
-        const int grow = m0 + q4 * 32 + lane;
         const bool ok = __all_sync(0xffffffffu, g_wait(g_smem(&b->done), 0, b, err));
         if (ok && !*(volatile int*)&b->abort) {
             g_fence_after();
@@ -238,35 +248,44 @@ __global__ void __launch_bounds__(kGThreads, 1)
             // 32 tokens x BN f32 of this warp, in 32-column boxes of 4 KB,
             // staged in the ring that the MMAs no longer read
             uint8_t* buf = smem + q4 * (32 * BN * 4);
-            float sq = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t o[32];
-                g_tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c, o);
-                uint8_t* box = buf + (c / 32) * 4096;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float* bj = bias + n0 + c + 4 * j;
-                    float4 v;
-                    v.x = __uint_as_float(o[4 * j + 0]) + __ldg(bj + 0);
-                    v.y = __uint_as_float(o[4 * j + 1]) + __ldg(bj + 1);
-                    v.z = __uint_as_float(o[4 * j + 2]) + __ldg(bj + 2);
-                    v.w = __uint_as_float(o[4 * j + 3]) + __ldg(bj + 3);
-                    sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
-                    // 16-byte chunk j of row `lane`, 128-byte swizzle
-                    *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+            for (int u = 0; u < halves; ++u) {
+                const int row0 = m0 + u * kGM + q4 * 32;  // this warp's first token
+                const int grow = row0 + lane;
+                if (u > 0) {
+                    // the previous half's stores have read the staging buffer
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    __syncwarp();
                 }
+                float sq = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t o[32];
+                    g_tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + u * BN + c, o);
+                    uint8_t* box = buf + (c / 32) * 4096;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float* bj = bias + n0 + c + 4 * j;
+                        float4 v;
+                        v.x = __uint_as_float(o[4 * j + 0]) + __ldg(bj + 0);
+                        v.y = __uint_as_float(o[4 * j + 1]) + __ldg(bj + 1);
+                        v.z = __uint_as_float(o[4 * j + 2]) + __ldg(bj + 2);
+                        v.w = __uint_as_float(o[4 * j + 3]) + __ldg(bj + 3);
+                        sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
+                        // 16-byte chunk j of row `lane`, 128-byte swizzle
+                        *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0 && row0 < tokens) {
+                    for (int c = 0; c < BN; c += 32)
+                        g_tma_store(&ty, g_smem(buf + (c / 32) * 4096), n0 + c, row0);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+                if (kind < 2 && grow < tokens) atomicAdd(ss + (size_t)grow * 2 + kind, sq);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
             __syncwarp();
-            if (lane == 0 && m0 + q4 * 32 < tokens) {
-                for (int c = 0; c < BN; c += 32)
-                    g_tma_store(&ty, g_smem(buf + (c / 32) * 4096), n0 + c, m0 + q4 * 32);
-                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-            }
-            __syncwarp();
-            if (kind < 2 && grow < tokens) atomicAdd(ss + (size_t)grow * 2 + kind, sq);
         }
     }
     g_fence_before();
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 1) {
         g_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"((uint32_t)BN)
+                     "r"((uint32_t)(kGHalves * BN))
                      : "memory");
     }
 }
@@ -291,7 +310,7 @@ cudaError_t launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const C
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    dim3 grid((tokens + kGM - 1) / kGM, 3 * dim / BN);
+    dim3 grid((tokens + kGM * kGHalves - 1) / (kGM * kGHalves), 3 * dim / BN);
     qkv_gemm_kernel<BN><<<grid, kGThreads, C::kSmem, s>>>(tx, tw, ty, bias, ss, tokens, dim, err);
     return cudaGetLastError();
 }

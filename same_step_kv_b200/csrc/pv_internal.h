@@ -106,7 +106,7 @@ cudaError_t launch_wait_timeout_probe(int* err, cudaStream_t s);
 
 // ----------------------------------------------------------------- Euler
 // q, k, v projection (pv_gemm.cu): y = x w^T + b in f32 and the q / k sums of
-// squares per token; tiles of 128 tokens x qkv_gemm_tile_n(dim) features.
+// squares per token; tiles of 256 tokens x qkv_gemm_tile_n(dim) features.
 int qkv_gemm_tile_n(int dim);
 cudaError_t launch_qkv_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
                             const float* bias, float* ss, int tokens, int dim, int* err,
