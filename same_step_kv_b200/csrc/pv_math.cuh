@@ -1,4 +1,8 @@
-// Device math shared by the attention kernel and its self-test entry point.
+// A software 2^x, kept with its self-test entry point (pv_selftest_exp2_poly).
+// Computing a share of the softmax exponentials with it instead of the XU
+// pipe measured slower at every share tried, so the attention kernel does not
+// use it; it stays tested against exp2f for when the balance of the pipes
+// changes.
 #pragma once
 
 #include <stdint.h>
@@ -25,11 +29,5 @@ __device__ __forceinline__ float exp2_poly(float x) {
     const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
-
-// Columns (of every 16) whose exponential is computed by exp2_poly.
-#ifndef PV_POLY_MASK
-#define PV_POLY_MASK 0x0000u  // none: measured faster on this kernel (see the sweep)
-#endif
-constexpr uint32_t kPolyMask = PV_POLY_MASK;
 
 }  // namespace pv
