@@ -58,12 +58,19 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant_
             const float4 k1 = __ldcs(reinterpret_cast<const float4*>(yq + dim + 4));
             const float4 v0 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim));
             const float4 v1 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim + 4));
+            // the gains as four 16-byte loads (f0 is a multiple of 8)
+            const float4 gq0 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0));
+            const float4 gq1 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0 + 4));
+            const float4 gk0 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0));
+            const float4 gk1 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0 + 4));
             const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
             const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            const float gqa[8] = {gq0.x, gq0.y, gq0.z, gq0.w, gq1.x, gq1.y, gq1.z, gq1.w};
+            const float gka[8] = {gk0.x, gk0.y, gk0.z, gk0.w, gk1.x, gk1.y, gk1.z, gk1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                qf[i] = qa[i] * sq * __ldg(p.g_q + f0 + i);
-                kf[i] = ka[i] * sk * __ldg(p.g_k + f0 + i);
+                qf[i] = qa[i] * sq * gqa[i];
+                kf[i] = ka[i] * sk * gka[i];
             }
             vv = make_uint4(pack(v0.x, v0.y), pack(v0.z, v0.w), pack(v1.x, v1.y), pack(v1.z, v1.w));
         } else {
