@@ -164,4 +164,9 @@ def test_qkv_rejects_bad_arguments(pv):
         pv.pv_qkv_rope_append(h, [0], 0, 0, x, w, f, f, f, 0.0, q_rot, ws, wsb)
     with pytest.raises(pv.PVError):
         pv.pv_qkv_rope_append(h, [0], 0, 0, x, 0, f, f, f, 1e-6, q_rot, ws, wsb)
+    # the gains are read as 16-byte vectors: a 4-byte offset is rejected
+    g_off = torch.zeros(385, device="cuda")[1:]
+    with pytest.raises(pv.PVError) as e:
+        pv.pv_qkv_rope_append(h, [0], 0, 0, x, w, f, g_off, f, 1e-6, q_rot, ws, wsb)
+    assert e.value.status == pv.PV_ERR_INVALID_ARG
     st.close()
