@@ -265,12 +265,15 @@ PV_API pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int
  * with n_sm SMs and a workspace of partial_slots split-KV slots (head_dim
  * 128), without launching anything: host only.  Items are (sequence, head,
  * 256-query block), each a run of ceil(n_k / 128) key tiles, laid out
- * query-block-major and end to end; CTA c processes the key tiles
- * [ranges[c], ranges[c + 1]) of that list.
+ * query-block-major and end to end.
  *  grid: CTAs; ranges: host array of at least min(n_sm, 160) + 1 entries.
- *  mode: 0 stream-K (equal ranges; split items are merged by the last CTA
- *  to arrive), 1 item-aligned with cost-balanced starts, 2 item-aligned
- *  with equal item counts (more than 65,535 items). */
+ *  mode 0, stream-K: CTA c processes the key tiles [ranges[c],
+ *    ranges[c + 1]) of the list (equal shares; an item split between CTAs is
+ *    merged by the last of them to arrive).
+ *  mode 1, whole items at run time: the sequences are put in decreasing
+ *    order of key tiles and each CTA takes the next whole item from a
+ *    counter until none is left (longest first); nothing is split.
+ *    ranges[0] = 0, ranges[grid] = the total key tiles, the others -1. */
 PV_API pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int heads, int n_sm,
                               int partial_slots, int* grid, int* mode, long long* ranges);
 

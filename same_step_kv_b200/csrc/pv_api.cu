@@ -981,21 +981,11 @@ pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int heads, in
         return fail(PV_ERR_CAPACITY, "no plan fits");
     *grid = p.grid;
     *mode = p.item_aligned;
-    // the key-tile range of every CTA, as the kernel derives it
-    std::vector<long long> item_start;
-    for (int i = 0; i < p.n_streams; ++i)
-        for (int k = 0; k < heads * p.st[i].n_qb; ++k)
-            item_start.push_back(p.st[i].cost0 + (long long)k * p.st[i].n_kt);
-    item_start.push_back(p.total);
-    for (int c = 0; c <= p.grid; ++c) {
-        if (p.item_aligned == 0) {
-            ranges[c] = (long long)c * p.total / p.grid;
-        } else {
-            const long long k = p.item_aligned == 1 ? (long long)p.first_item[c]
-                                                    : (long long)c * p.n_items / p.grid;
-            ranges[c] = item_start[std::min<long long>(k, p.n_items)];
-        }
-    }
+    // stream-K: the key-tile range of every CTA, as the kernel derives it;
+    // whole items at run time: no fixed ranges, only the two ends
+    for (int c = 0; c <= p.grid; ++c)
+        ranges[c] = p.item_aligned == 0 ? (long long)c * p.total / p.grid
+                                        : (c == 0 ? 0 : c == p.grid ? p.total : -1);
     return PV_OK;
 }
 

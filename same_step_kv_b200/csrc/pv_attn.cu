@@ -41,6 +41,7 @@ constexpr int kRegsLow = 96;    // warpgroup 0 after setmaxnreg.dec
 constexpr int kRegsHigh = 200;  // softmax warpgroups after setmaxnreg.inc
 static_assert(kRegsLow * 128 + 2 * kRegsHigh * 128 <= 168 * kThreads, "register split");
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+constexpr int kRing = 4;  // slots of the run-time item hand-out
 
 template <int D>
 struct Cfg {
@@ -57,7 +58,7 @@ struct Cfg {
     static constexpr uint32_t kColsO = 256;
 };
 
-struct Bars {  // 264 bytes, inside the 512 reserved after the tiles
+struct Bars {  // 344 bytes, inside the 512 reserved after the tiles
     uint64_t q_full;
     uint64_t q_empty;
     uint64_t o_empty[2];
@@ -70,10 +71,14 @@ struct Bars {  // 264 bytes, inside the 512 reserved after the tiles
     uint64_t mma_done;
     uint64_t kv_full[8];
     uint64_t rel[8];      // release events: the K/V tiles they free may be overwritten
+    uint64_t ring_full[kRing];   // items handed out at run time (item_grab / item_take)
+    uint64_t ring_empty[kRing];
+    int ring[kRing];
     uint32_t tmem_base;
     int abort;
     int last[2];
 };
+static_assert(sizeof(Bars) <= 512, "barriers beyond their reserved bytes");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -290,18 +295,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 
 // ----------------------------------------------------------------- schedule
-// CTA c owns the key tiles [bound(c), bound(c+1)) of the launch's item list
-// (see pv_plan.cu).  A segment is the part of one item inside that range.
+// Stream-K: CTA c owns the key tiles [bound(c), bound(c+1)) of the launch's
+// item list (see pv_plan.cu).  A segment is the part of one item inside that
+// range.  Whole items at run time: every segment is a whole item.
 __device__ __forceinline__ long long bound(const AttnParams& p, int c) {
-    if (!p.item_aligned) return (long long)c * p.total / p.grid;
-    // whole items: CTA c starts at item first_item[c] (balanced by the host),
-    // or at item c * n_items / grid when the table cannot hold the indices
-    const int k = p.item_aligned == 1 ? (int)p.first_item[c]
-                                      : (int)((long long)c * p.n_items / p.grid);
-    int i = 0;
-    while (i + 1 < p.n_streams && p.st[i + 1].item0 <= k) ++i;
-    if (k >= p.n_items) return p.total;
-    return p.st[i].cost0 + (long long)(k - p.st[i].item0) * p.st[i].n_kt;
+    return (long long)c * p.total / p.grid;
 }
 // The CTA whose range holds key tile x.
 __device__ __forceinline__ int cta_of(const AttnParams& p, long long x) {
@@ -317,9 +315,40 @@ struct Seg {
     int which;     // 0: this CTA's first segment, 1: a later one
 };
 
+// Item li of stream si, key tiles [kt0, kt0 + n).  Items are laid out
+// query-block-major: with a grid that is a multiple of n_qb, the CTAs
+// working on one head's query blocks walk the same key tiles at the same
+// time and share them through L2.
+__device__ __forceinline__ void make_seg(const AttnParams& p, int si, int li, int kt0, int n,
+                                         Seg& g) {
+    const AttnStreamDesc& s = p.st[si];
+    g.si = si;
+    g.kt0 = kt0;
+    g.n = n;
+    g.qb = li / p.heads;
+    g.head = li - g.qb * p.heads;
+    g.item = s.item0 + li;
+    g.i0 = s.cost0 + (long long)li * s.n_kt;
+    g.q0 = g.qb * kQBlock;
+    g.rows[0] = min(kQRows, s.n_q - g.q0);
+    g.rows[1] = max(0, min(kQRows, s.n_q - g.q0 - kQRows));
+}
+
+// The whole item `item` as one segment (items handed out at run time).
+__device__ __forceinline__ void item_seg(const AttnParams& p, int item, Seg& g) {
+    int i = 0;
+    while (i + 1 < p.n_streams && p.st[i + 1].item0 <= item) ++i;
+    make_seg(p, i, item - p.st[i].item0, 0, p.st[i].n_kt, g);
+    g.c_first = blockIdx.x;
+    g.nseg = 1;
+    g.which = 0;
+}
+
 struct SegIter {
     long long pos, end;
-    __device__ SegIter(const AttnParams& p) : pos(bound(p, blockIdx.x)), end(bound(p, blockIdx.x + 1)) {}
+    __device__ SegIter(const AttnParams& p)
+        : pos(p.item_aligned ? 0 : bound(p, blockIdx.x)),
+          end(p.item_aligned ? 0 : bound(p, blockIdx.x + 1)) {}
     __device__ bool next(const AttnParams& p, Seg& g) {
         if (pos >= end) return false;
         int i = 0;
@@ -327,34 +356,48 @@ struct SegIter {
         const AttnStreamDesc& s = p.st[i];
         const long long off = pos - s.cost0;
         const int li = (int)(off / s.n_kt);
-        g.si = i;
-        g.kt0 = (int)(off - (long long)li * s.n_kt);
         const long long i0 = s.cost0 + (long long)li * s.n_kt;   // the item's key-tile range
         const long long i1 = i0 + s.n_kt;
         const long long e = i1 < end ? i1 : end;
-        g.n = (int)(e - pos);
+        make_seg(p, i, li, (int)(off - (long long)li * s.n_kt), (int)(e - pos), g);
         g.which = pos == bound(p, blockIdx.x) ? 0 : 1;
-        // items are laid out query-block-major: with a grid that is a multiple
-        // of n_qb, the CTAs working on one head's query blocks then walk the
-        // same key tiles at the same time and share them through L2
-        g.qb = li / p.heads;
-        g.head = li - g.qb * p.heads;
-        g.item = s.item0 + li;
-        g.i0 = i0;
-        if (p.item_aligned) {
-            g.c_first = blockIdx.x;
-            g.nseg = 1;
-        } else {
-            g.c_first = cta_of(p, i0);
-            g.nseg = cta_of(p, i1 - 1) - g.c_first + 1;
-        }
-        g.q0 = g.qb * kQBlock;
-        g.rows[0] = min(kQRows, s.n_q - g.q0);
-        g.rows[1] = max(0, min(kQRows, s.n_q - g.q0 - kQRows));
+        g.c_first = cta_of(p, i0);
+        g.nseg = cta_of(p, i1 - 1) - g.c_first + 1;
         pos = e;
         return true;
     }
 };
+
+// Items handed out at run time.  The producer thread takes the next item
+// index from counters[0] and passes it to the MMA warp and the eight softmax
+// warps through a ring of kRing shared-memory slots; -1 ends the list.
+// Slot k is written once the consumers have all released slot k - kRing.
+__device__ bool item_grab(const AttnParams& p, Bars* b, int& k, Seg& g, bool& ok) {
+    const int s = k % kRing;
+    if (k >= kRing && !(ok = mbar_wait(smem_u32(&b->ring_empty[s]), ((k / kRing) - 1) & 1, b, p.err)))
+        return false;
+    int item = atomicAdd(p.counters, 1);
+    if (item >= p.n_items) item = -1;
+    *(volatile int*)&b->ring[s] = item;
+    mbar_arrive(smem_u32(&b->ring_full[s]));  // release: the slot's value is visible
+    ++k;
+    if (item < 0) return false;
+    item_seg(p, item, g);
+    return true;
+}
+// Warp-wide: the next slot of the ring.
+__device__ bool item_take(const AttnParams& p, Bars* b, int& k, Seg& g, bool& ok) {
+    const int s = k % kRing;
+    ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->ring_full[s]), (k / kRing) & 1, b, p.err));
+    if (!ok) return false;
+    const int item = *(volatile int*)&b->ring[s];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->ring_empty[s]));
+    ++k;
+    if (item < 0) return false;
+    item_seg(p, item, g);
+    return true;
+}
 
 // Partial slot of CTA c's part of an item starting at key tile i0, tile X.
 __device__ __forceinline__ size_t part_slot(const AttnParams& p, int c, long long i0, int X) {
@@ -372,9 +415,10 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     int ev0 = 0;              // first release event of the current segment
     int stage_ev[C::kStages]; // release event of the tile in each stage
     bool ok = true;
+    int rk = 0;  // ring slots written
     SegIter it(p);
     Seg g;
-    while (ok && it.next(p, g)) {
+    while (ok && (p.item_aligned ? item_grab(p, b, rk, g, ok) : it.next(p, g))) {
         const AttnStreamDesc& s = p.st[g.si];
         const int ntile = g.rows[1] > 0 ? 2 : 1;
         // the previous segment's S products are done with the Q tiles
@@ -476,9 +520,10 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
         pv(X, stage, true, kKeyTile / 32);
         return true;
     };
+    int rk = 0;  // ring slots taken
     SegIter it(p);
     Seg g;
-    while (ok && it.next(p, g)) {
+    while (ok && (p.item_aligned ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
         const bool hasB = g.rows[1] > 0;
         if (!(ok = wspin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
         ++qseg;
@@ -717,9 +762,10 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
     int oc = 0;   // segments finished, for the o_full phase
     int ec = 0;   // split epilogues, for the ep_in / ep_out phases
     bool ok = true;
+    int rk = 0;  // ring slots taken
     SegIter it(p);
     Seg g;
-    while (ok && it.next(p, g)) {
+    while (ok && (p.item_aligned ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
         if (g.rows[X] == 0) continue;  // this segment has no query tile X
         const AttnStreamDesc& s = p.st[g.si];
         float m = -INFINITY;  // maximum applied to the exponentials, log2 units
@@ -891,6 +937,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&b->mma_done), 1);
         for (int i = 0; i < C::kStages; ++i) mbar_init(smem_u32(&b->kv_full[i]), 1);
         for (int i = 0; i < 8; ++i) mbar_init(smem_u32(&b->rel[i]), 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(smem_u32(&b->ring_full[i]), 1);
+            mbar_init(smem_u32(&b->ring_empty[i]), 9);  // the MMA warp and 8 softmax warps
+        }
         b->abort = 0;
         b->last[0] = b->last[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -920,6 +970,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    if (p.item_aligned && threadIdx.x == 0) {
+        // every CTA has stopped taking items once it gets here: the last one
+        // to arrive returns the hand-out counter to zero for the next launch
+        __threadfence();
+        if (atomicAdd(p.counters + 1, 1) == p.grid - 1) {
+            p.counters[0] = 0;
+            p.counters[1] = 0;
+        }
+    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u)

@@ -73,9 +73,10 @@ struct AttnStreamDesc {
 };
 
 // One launch is a list of items (head, query block) of all streams, each
-// costing n_kt key tiles, laid end to end; CTA c of `grid` processes one
-// contiguous range of that list (pv_plan.cu chooses the ranges).  The whole
-// struct plus three tensor maps stays under 4 KB of kernel parameters.
+// costing n_kt key tiles, laid end to end.  Under stream-K, CTA c of `grid`
+// processes one contiguous range of that list; otherwise the CTAs take whole
+// items one at a time (pv_plan.cu chooses).  The whole struct plus four
+// tensor maps stays under 4 KB of kernel parameters.
 struct AttnParams {
     bf16* out;
     float* lse;
@@ -87,11 +88,10 @@ struct AttnParams {
     float scale_log2;    // log2(e) / sqrt(D)
     int n_streams;
     int grid;            // CTAs of the launch
-    int item_aligned;    // 0: stream-K; 1, 2: CTA ranges end on item boundaries (no partial
-                         // results), at first_item[] (1) or at equal item counts (2)
+    int item_aligned;    // 0: stream-K; 1: whole items handed out at run time, in
+                         // list order, from counters[0] (no partial results)
     int n_items;         // items of all streams
     long long total;     // key tiles of all items
-    uint16_t first_item[kMaxGrid + 1];  // item_aligned == 1: CTA c's first item
     AttnStreamDesc st[PV_MAX_STREAMS];
 };
 
@@ -131,11 +131,12 @@ bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, 
 // Records a failure for pv_last_error() and returns code.
 pv_status report_error(pv_status code, const char* msg);
 
-// Stream-K plan for one attention launch: fills n_qb, n_kt, item0, cost0 of
-// every stream and grid, total, n_items, item_aligned of p.  Returns the
-// number of CTAs, or -1 when the counters (2 per item) do not fit.  When the
-// partial slots (4 per CTA) do not suffice for one CTA per SM, the CTAs take
-// whole items instead (item_aligned) and need none.
+// Work plan for one attention launch: fills n_qb, n_kt, item0, cost0 of
+// every stream and grid, total, n_items, item_aligned of p (and may reorder
+// p.st).  Returns the number of CTAs, or -1 when the counters (one per item,
+// at least two) do not fit.  Long items run stream-K; short items, or a
+// workspace without room for the partial slots (4 per CTA), get whole items
+// handed out at run time instead.
 int plan_attention(AttnParams& p, int n_sm, int part_capacity, int cnt_capacity);
 
 }  // namespace pv
