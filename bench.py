@@ -473,6 +473,125 @@ def run_sampler(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+N_CHUNKS = 28       # one-frame chunks after the 3-frame first chunk: 31 latent frames
+POOL = 4            # distinct synthetic q, k, v sets cycled through the schedule
+
+
+def run_schedule(args, rank, world, local):
+    """The whole generation schedule of one stream: the first chunk (3 frames,
+    4 steps), the sigma = 0 sink pass, then N_CHUNKS one-frame chunks of 4
+    steps, each step a rope/append + chunk attention per layer and an Euler
+    update of the chunk's latent.  One bench step = the whole schedule."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    NL = args.layers
+    cfg = pv.make_config(NL, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
+    store = pv.KVStore(cfg, device=dev)
+    h = store.handle
+    big = [synth.chunk_qkv(rank, 0, i, 0, 3 * T, HEADS, D, dev) for i in range(POOL)]
+    small = [synth.chunk_qkv(rank, 1, i, 0, T, HEADS, D, dev) for i in range(POOL)]
+    q_rot = torch.empty(HEADS * 3 * T * D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(3 * T, HEADS, D, dtype=torch.bfloat16, device=dev)
+    x = synth.latent(rank, 3 + N_CHUNKS, 48, 44, 80, dev).reshape(-1)
+    vel = synth.velocity(rank, 0, 0, 3 * LATENT, dev)
+    sig = [1.0, 0.75, 0.5, 0.25, 0.0]
+    new_state = pv.pv_kv_state()
+    new_state.phase, new_state.chunk = pv.PV_PHASE_NEW, -1
+
+    def keys(j):  # key count of chunk j >= 1 at any step
+        return 3 * T + min(j, R) * T
+
+    flops = 4 * NL * (4 + 1) * (3 * T) ** 2 * HEADS * D
+    flops += sum(4 * NL * 4 * T * keys(j) * HEADS * D for j in range(1, N_CHUNKS + 1))
+    attn_ev = []
+
+    def layer_pass(j, s, n, inputs, record):
+        step_arg = pv.PV_STEP_SINK if s is None else s
+        for layer in range(NL):
+            q, k, v = inputs[(j * 7 + (0 if s is None else s) * 3 + layer) % POOL]
+            pv.pv_rope_append(h, [0], layer, step_arg, q, k, v, q_rot, cs)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+            pv.pv_chunk_attn(h, [0], layer, step_arg, q_rot[: HEADS * n * D], out[:n], None, cs)
+            if record:
+                e1.record(cs)
+                attn_ev.append((e0, e1))
+
+    def step(record):
+        pv.pv_kv_set_state(h, 0, new_state)
+        pv.pv_kv_begin_chunk(h, 0, 3)
+        for s in range(4):
+            layer_pass(0, s, 3 * T, big, record)
+            pv.pv_euler_step(x[: 3 * LATENT], vel, 3 * LATENT, sig[s + 1] - sig[s], cs)
+        pv.pv_kv_begin_sink(h, 0)
+        layer_pass(0, None, 3 * T, big, record)
+        for j in range(1, N_CHUNKS + 1):
+            pv.pv_kv_begin_chunk(h, 0, 1)
+            xj = x[(2 + j) * LATENT:(3 + j) * LATENT]
+            for s in range(4):
+                layer_pass(j, s, T, small, record)
+                pv.pv_euler_step(xj, vel[:LATENT], LATENT, sig[s + 1] - sig[s], cs)
+
+    # the schedule timed without per-launch events (3,510 pairs would add to
+    # it), then one more pass with them for the attention kernel's own time
+    ms_step, clocks = timed_steps(lambda record: step(False), args, local, world, cs)
+    step(True)
+    torch.cuda.synchronize()
+    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev)
+    # e2e: the latent from pinned host memory and back, every input set too
+    hx = x.cpu().pin_memory()
+    hpool = [[t.cpu().pin_memory() for t in qkv] for qkv in big + small]
+    dpool = big + small
+
+    def e2e_step(record):
+        x.copy_(hx, non_blocking=True)
+        for dst, src in zip(dpool, hpool):
+            for a, b in zip(dst, src):
+                a.copy_(b, non_blocking=True)
+        step(False)
+        hx.copy_(x, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    h2d = x.numel() * 4 + sum(t.numel() * 2 for qkv in dpool for t in qkv)
+    launches = 2 * NL * (4 + 1 + 4 * N_CHUNKS) + 4 * (1 + N_CHUNKS)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        line = {
+            "metric": "chunk-attention TFLOP/s over the whole generation schedule; latent frames/s",
+            "value": flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"whole schedule: first chunk 3 x 880 tokens (4 steps) + sink "
+                                   f"pass + {N_CHUNKS} chunks x 880 tokens x 4 steps, ring {R}, "
+                                   f"24x128, {NL} layers, Euler on 48x44x80 per frame",
+                       "l2": "K/V store of %.1f GB, no flush" % (store.kv_bytes / 1e9)},
+            "latent_frames_per_s": world * (3 + N_CHUNKS) / (ms_step * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{src} bf16_tflops_sustained",
+                         "kernel": "attn_kernel<128> (every pv_chunk_attn of the schedule)",
+                         "traffic": None, "ms_attention_per_step": attn_ms},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": x.numel() * 4},
+            "gpu_launches": args.steps * launches, "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    store.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -484,13 +603,15 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers per step (30 in the profile; fewer only for small ncu captures)")
     ap.add_argument("--workload", default="step",
-                    choices=["step", "cross_attn", "sampler", "qkv"],
-                    help="step: the same-step KV chunk step (default); cross_attn, sampler, "
-                         "qkv: the cross-attention, sampler-variant and q/k/v projection "
-                         "kernels on their own")
+                    choices=["step", "schedule", "cross_attn", "sampler", "qkv"],
+                    help="step: the same-step KV chunk step (default); schedule: the whole "
+                         "29-chunk generation of one stream; cross_attn, sampler, qkv: the "
+                         "cross-attention, sampler-variant and q/k/v projection kernels on "
+                         "their own")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"step": 100, "cross_attn": 400, "sampler": 2000, "qkv": 50}[args.workload]
+        args.steps = {"step": 100, "schedule": 3, "cross_attn": 400, "sampler": 2000,
+                      "qkv": 50}[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -501,7 +622,8 @@ def main():
         run_reference(args, rank)
         return
     if args.workload != "step":
-        {"cross_attn": run_cross_attn, "sampler": run_sampler, "qkv": run_qkv}[args.workload](
+        {"schedule": run_schedule, "cross_attn": run_cross_attn, "sampler": run_sampler,
+         "qkv": run_qkv}[args.workload](
             args, rank, world, local)
         if world > 1:
             import torch.distributed as dist
