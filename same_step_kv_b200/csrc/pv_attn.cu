@@ -71,12 +71,12 @@ struct Bars {  // 344 bytes, inside the 512 reserved after the tiles
     uint64_t mma_done;
     uint64_t kv_full[8];
     uint64_t rel[8];      // release events: the K/V tiles they free may be overwritten
-    uint64_t ring_full[kRing];   // items handed out at run time (item_grab / item_take)
-    uint64_t ring_empty[kRing];
-    int ring[kRing];
     uint32_t tmem_base;
     int abort;
     int last[2];
+    uint64_t ring_full[kRing];   // items handed out at run time (item_grab / item_take)
+    uint64_t ring_empty[kRing];
+    int ring[kRing];
 };
 static_assert(sizeof(Bars) <= 512, "barriers beyond their reserved bytes");
 
@@ -315,40 +315,30 @@ struct Seg {
     int which;     // 0: this CTA's first segment, 1: a later one
 };
 
-// Item li of stream si, key tiles [kt0, kt0 + n).  Items are laid out
-// query-block-major: with a grid that is a multiple of n_qb, the CTAs
-// working on one head's query blocks walk the same key tiles at the same
-// time and share them through L2.
-__device__ __forceinline__ void make_seg(const AttnParams& p, int si, int li, int kt0, int n,
-                                         Seg& g) {
-    const AttnStreamDesc& s = p.st[si];
-    g.si = si;
-    g.kt0 = kt0;
-    g.n = n;
+// The whole item `item` as one segment (items handed out at run time).
+__device__ __forceinline__ void item_seg(const AttnParams& p, int item, Seg& g) {
+    int i = 0;
+    while (i + 1 < p.n_streams && p.st[i + 1].item0 <= item) ++i;
+    const AttnStreamDesc& s = p.st[i];
+    const int li = item - s.item0;
+    g.si = i;
+    g.kt0 = 0;
+    g.n = s.n_kt;
     g.qb = li / p.heads;
     g.head = li - g.qb * p.heads;
-    g.item = s.item0 + li;
+    g.item = item;
     g.i0 = s.cost0 + (long long)li * s.n_kt;
+    g.c_first = blockIdx.x;
+    g.nseg = 1;
+    g.which = 0;
     g.q0 = g.qb * kQBlock;
     g.rows[0] = min(kQRows, s.n_q - g.q0);
     g.rows[1] = max(0, min(kQRows, s.n_q - g.q0 - kQRows));
 }
 
-// The whole item `item` as one segment (items handed out at run time).
-__device__ __forceinline__ void item_seg(const AttnParams& p, int item, Seg& g) {
-    int i = 0;
-    while (i + 1 < p.n_streams && p.st[i + 1].item0 <= item) ++i;
-    make_seg(p, i, item - p.st[i].item0, 0, p.st[i].n_kt, g);
-    g.c_first = blockIdx.x;
-    g.nseg = 1;
-    g.which = 0;
-}
-
 struct SegIter {
     long long pos, end;
-    __device__ SegIter(const AttnParams& p)
-        : pos(p.item_aligned ? 0 : bound(p, blockIdx.x)),
-          end(p.item_aligned ? 0 : bound(p, blockIdx.x + 1)) {}
+    __device__ SegIter(const AttnParams& p) : pos(bound(p, blockIdx.x)), end(bound(p, blockIdx.x + 1)) {}
     __device__ bool next(const AttnParams& p, Seg& g) {
         if (pos >= end) return false;
         int i = 0;
@@ -356,13 +346,25 @@ struct SegIter {
         const AttnStreamDesc& s = p.st[i];
         const long long off = pos - s.cost0;
         const int li = (int)(off / s.n_kt);
+        g.si = i;
+        g.kt0 = (int)(off - (long long)li * s.n_kt);
         const long long i0 = s.cost0 + (long long)li * s.n_kt;   // the item's key-tile range
         const long long i1 = i0 + s.n_kt;
         const long long e = i1 < end ? i1 : end;
-        make_seg(p, i, li, (int)(off - (long long)li * s.n_kt), (int)(e - pos), g);
+        g.n = (int)(e - pos);
         g.which = pos == bound(p, blockIdx.x) ? 0 : 1;
+        // items are laid out query-block-major: with a grid that is a multiple
+        // of n_qb, the CTAs working on one head's query blocks then walk the
+        // same key tiles at the same time and share them through L2
+        g.qb = li / p.heads;
+        g.head = li - g.qb * p.heads;
+        g.item = s.item0 + li;
+        g.i0 = i0;
         g.c_first = cta_of(p, i0);
         g.nseg = cta_of(p, i1 - 1) - g.c_first + 1;
+        g.q0 = g.qb * kQBlock;
+        g.rows[0] = min(kQRows, s.n_q - g.q0);
+        g.rows[1] = max(0, min(kQRows, s.n_q - g.q0 - kQRows));
         pos = e;
         return true;
     }
@@ -406,7 +408,7 @@ __device__ __forceinline__ size_t part_slot(const AttnParams& p, int c, long lon
 }
 
 // ----------------------------------------------------------------- roles
-template <int D>
+template <int D, bool kRun>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const AttnParams& p, uint8_t* smem, Bars* b) {
     using C = Cfg<D>;
@@ -418,7 +420,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     int rk = 0;  // ring slots written
     SegIter it(p);
     Seg g;
-    while (ok && (p.item_aligned ? item_grab(p, b, rk, g, ok) : it.next(p, g))) {
+    while (ok && (kRun ? item_grab(p, b, rk, g, ok) : it.next(p, g))) {
         const AttnStreamDesc& s = p.st[g.si];
         const int ntile = g.rows[1] > 0 ? 2 : 1;
         // the previous segment's S products are done with the Q tiles
@@ -470,7 +472,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     }
 }
 
-template <int D>
+template <int D, bool kRun>
 __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t tmem) {
     using C = Cfg<D>;
     // every lane waits; the vote reconverges the warp before the next issue
@@ -523,7 +525,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     int rk = 0;  // ring slots taken
     SegIter it(p);
     Seg g;
-    while (ok && (p.item_aligned ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
+    while (ok && (kRun ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
         const bool hasB = g.rows[1] > 0;
         if (!(ok = wspin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
         ++qseg;
@@ -745,7 +747,7 @@ __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, i
     if (row_ok && lse_dst) *lse_dst = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
-template <int D>
+template <int D, bool kRun>
 __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uint8_t* smem,
                                  Bars* b, uint32_t tmem, int X) {
     using C = Cfg<D>;
@@ -765,7 +767,7 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
     int rk = 0;  // ring slots taken
     SegIter it(p);
     Seg g;
-    while (ok && (p.item_aligned ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
+    while (ok && (kRun ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
         if (g.rows[X] == 0) continue;  // this segment has no query tile X
         const AttnStreamDesc& s = p.st[g.si];
         float m = -INFINITY;  // maximum applied to the exponentials, log2 units
@@ -910,7 +912,9 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
     __syncwarp();
 }
 
-template <int D>
+// kRun: whole items handed out at run time (AttnParams::item_aligned == 1);
+// otherwise stream-K.  Two instantiations, so that each keeps its own code.
+template <int D, bool kRun>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -960,17 +964,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
         if (warp == 0) {
-            if (lane_id == 0) producer<D>(&tq, &tk, &tv, p, smem, b);
+            if (lane_id == 0) producer<D, kRun>(&tq, &tk, &tv, p, smem, b);
         } else if (warp == 1) {
-            mma_issuer<D>(p, smem, b, tmem);  // the whole warp; one elected lane issues
+            mma_issuer<D, kRun>(p, smem, b, tmem);  // the whole warp; one elected lane issues
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-        softmax_epilogue<D>(p, &to, smem, b, tmem, warp / 4 - 1);
+        softmax_epilogue<D, kRun>(p, &to, smem, b, tmem, warp / 4 - 1);
     }
     tc_fence_before();
     __syncthreads();
-    if (p.item_aligned && threadIdx.x == 0) {
+    if (kRun && threadIdx.x == 0) {
         // every CTA has stopped taking items once it gets here: the last one
         // to arrive returns the hand-out counter to zero for the next launch
         __threadfence();
@@ -986,18 +990,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, bool kRun>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& to, const AttnParams& p, cudaStream_t s) {
     using C = Cfg<D>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kRun>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    attn_kernel<D><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, to, p);
+    attn_kernel<D, kRun><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -1027,8 +1031,11 @@ static_assert(sizeof(AttnParams) + 4 * sizeof(CUtensorMap) <= 4096,
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& to, const AttnParams& p, cudaStream_t s) {
     if (p.grid <= 0 || p.total <= 0) return cudaErrorInvalidValue;
-    if (p.head_dim == 128) return launch_d<128>(tq, tk, tv, to, p, s);
-    if (p.head_dim == 64) return launch_d<64>(tq, tk, tv, to, p, s);
+    const bool run = p.item_aligned != 0;
+    if (p.head_dim == 128)
+        return run ? launch_d<128, true>(tq, tk, tv, to, p, s) : launch_d<128, false>(tq, tk, tv, to, p, s);
+    if (p.head_dim == 64)
+        return run ? launch_d<64, true>(tq, tk, tv, to, p, s) : launch_d<64, false>(tq, tk, tv, to, p, s);
     return cudaErrorInvalidValue;
 }
 
