@@ -473,6 +473,190 @@ def run_sampler(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+DENSE_FRAMES = 21   # whole-video attention: 21 latent frames = 18,480 tokens
+N_STREAMS = 8       # batched serving: streams in one launch
+
+
+def run_dense(args, rank, world, local):
+    """Full bidirectional attention over a whole latent video (21 frames x 880
+    tokens attending to all 18,480), 24 x 128, 3D RoPE at frames 0..20: per
+    layer one pv_rope_dense and one pv_attn_dense."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    n = DENSE_FRAMES * T
+    cfg = pv.make_config(1, HEADS, D, W, HH, ring_slots=R, max_streams=1, max_frames=64)
+    store = pv.KVStore(cfg, device=dev)
+    q, k, v = synth.chunk_qkv(rank, 0, 0, 0, n, HEADS, D, dev)
+    q_rot = torch.empty(HEADS, n, D, dtype=torch.bfloat16, device=dev)
+    k_rot, v_hm = torch.empty_like(q_rot), torch.empty_like(q_rot)
+    out = torch.empty(n, HEADS, D, dtype=torch.bfloat16, device=dev)
+    wsb = pv.pv_attn_dense_ws_bytes(n, n, HEADS, D)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+    ev = []
+
+    def step(record):
+        pv.pv_rope_dense(store.handle, n, 0, q, k, v, q_rot, k_rot, v_hm, cs)
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(cs)
+        pv.pv_attn_dense(q_rot, k_rot, v_hm, n, n, HEADS, D, out, None, ws, wsb, cs)
+        if record:
+            e1.record(cs)
+            ev.append((e0, e1))
+
+    ms_step, clocks = timed_steps(step, args, local, world, cs)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = 4 * n * n * HEADS * D
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step(record):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step(False)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        achieved = flops / (launch_ms * 1e-3) / 1e12
+        line = {
+            "metric": "dense video attention TFLOP/s (18,480 x 18,480, 24x128, RoPE + attention)",
+            "value": flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"whole video: {DENSE_FRAMES} latent frames x 880 tokens, "
+                                   "all-to-all, 24x128, one layer per step",
+                       "l2": "q, k, v of 0.34 GB per step (larger than L2), no flush"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": f"{src} bf16_tflops_sustained",
+                         "kernel": "attn_kernel<128> (pv_attn_dense)", "traffic": None,
+                         "ms_per_launch": launch_ms},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * n * HEADS * D * 2,
+                    "d2h_bytes_per_step": n * HEADS * D * 2},
+            "gpu_launches": 2 * args.steps, "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    store.close()
+
+
+def run_multistream(args, rank, world, local):
+    """Batched serving: N_STREAMS streams, each at its own steady chunk with a
+    seeded ragged ring fill (0..18 earlier chunks), one pv_rope_append and one
+    pv_chunk_attn over all streams per layer, 30 layers, then the Euler update
+    of the streams' latent frames."""
+    import torch
+    from same_step_kv_b200 import pv, synth
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    cs = torch.cuda.current_stream()
+    NL = args.layers
+    fills = synth.ragged_fills(N_STREAMS, R, seed=rank)
+    # one step buffer per layer and stream (the step timed is one denoising
+    # step): 30 layers x 8 streams x 18,480 keys is 54.5 GB of K/V
+    cfg = pv.make_config(NL, HEADS, D, W, HH, ring_slots=R, steps=1, max_streams=N_STREAMS,
+                         max_frames=64)
+    store = pv.KVStore(cfg, device=dev)
+    h = store.handle
+    Kr, Vr = store.k_region(), store.v_region()
+    n_keys = []
+    for i, f in enumerate(fills):
+        st = pv.pv_kv_state()
+        st.phase, st.chunk = pv.PV_PHASE_STEADY, f + 1
+        pv.pv_kv_set_state(h, i, st)
+        nk = pv.pv_kv_get_state(h, i).n_keys
+        n_keys.append(nk)
+        kf, vf = synth.store_fill(rank * N_STREAMS + i, 0, 0, HEADS, nk, D, dev)
+        for layer in range(NL):
+            Kr[layer, 0, i, :, :nk] = kf
+            Vr[layer, 0, i, :, :nk] = vf
+        del kf, vf
+    streams = list(range(N_STREAMS))
+    tok = N_STREAMS * T
+    qkv = [synth.chunk_qkv(rank, 1000 + layer, 0, layer, tok, HEADS, D, dev) for layer in range(NL)]
+    q_rot = torch.empty(HEADS * tok * D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(tok, HEADS, D, dtype=torch.bfloat16, device=dev)
+    x = synth.latent(rank, N_STREAMS, 48, 44, 80, dev).reshape(-1)
+    vel = synth.velocity(rank, 0, 0, N_STREAMS * LATENT, dev)
+    ev = []
+
+    def step(record):
+        for layer in range(NL):
+            q, k, v = qkv[layer]
+            pv.pv_rope_append(h, streams, layer, 0, q, k, v, q_rot, cs)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(cs)
+            pv.pv_chunk_attn(h, streams, layer, 0, q_rot, out, None, cs)
+            if record:
+                e1.record(cs)
+                ev.append((e0, e1))
+        pv.pv_euler_step(x, vel, N_STREAMS * LATENT, -0.25, cs)
+
+    ms_step, clocks = timed_steps(step, args, local, world, cs)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = sum(4 * T * nk * HEADS * D for nk in n_keys)
+    hq = [[t.cpu().pin_memory() for t in qkv[layer]] for layer in range(NL)]
+    dq = [torch.empty_like(t) for t in qkv[0]]
+    hx = x.cpu().pin_memory()
+
+    def e2e_step(record):
+        x.copy_(hx, non_blocking=True)
+        for layer in range(NL):
+            for a, b in zip(dq, hq[layer]):
+                a.copy_(b, non_blocking=True)
+            pv.pv_rope_append(h, streams, layer, 0, dq[0], dq[1], dq[2], q_rot, cs)
+            pv.pv_chunk_attn(h, streams, layer, 0, q_rot, out, None, cs)
+        pv.pv_euler_step(x, vel, N_STREAMS * LATENT, -0.25, cs)
+        hx.copy_(x, non_blocking=True)
+
+    e2e_ms, _ = timed_steps(e2e_step, args, local, world, cs)
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        achieved = flops / (launch_ms * 1e-3) / 1e12
+        line = {
+            "metric": "batched chunk-attention TFLOP/s; latent frames/s per denoise step",
+            "value": NL * flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{N_STREAMS} streams x 880 tokens, ragged ring fills {fills}, "
+                                   f"24x128, {NL} layers + Euler",
+                       "keys_per_stream": n_keys,
+                       "l2": "K/V working set larger than L2, no flush"},
+            "latent_frames_per_s": world * N_STREAMS / (ms_step * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": f"{src} bf16_tflops_sustained",
+                         "kernel": "attn_kernel<128> (pv_chunk_attn, 8 streams)", "traffic": None,
+                         "ms_per_launch": launch_ms},
+            "e2e": {"value": NL * flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": NL * 3 * tok * HEADS * D * 2 + x.numel() * 4,
+                    "d2h_bytes_per_step": x.numel() * 4},
+            "gpu_launches": args.steps * (2 * NL + 1), "clocks": clocks, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    store.close()
+
+
 N_CHUNKS = 28       # one-frame chunks after the 3-frame first chunk: 31 latent frames
 POOL = 4            # distinct synthetic q, k, v sets cycled through the schedule
 
@@ -603,15 +787,18 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layers per step (30 in the profile; fewer only for small ncu captures)")
     ap.add_argument("--workload", default="step",
-                    choices=["step", "schedule", "cross_attn", "sampler", "qkv"],
+                    choices=["step", "schedule", "dense", "multistream", "cross_attn", "sampler",
+                             "qkv"],
                     help="step: the same-step KV chunk step (default); schedule: the whole "
-                         "29-chunk generation of one stream; cross_attn, sampler, qkv: the "
+                         "29-chunk generation of one stream; dense: whole-video attention "
+                         "(18,480 tokens); multistream: 8 streams at ragged ring fills in "
+                         "one launch; cross_attn, sampler, qkv: the "
                          "cross-attention, sampler-variant and q/k/v projection kernels on "
                          "their own")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"step": 100, "schedule": 3, "cross_attn": 400, "sampler": 2000,
-                      "qkv": 50}[args.workload]
+        args.steps = {"step": 100, "schedule": 3, "dense": 20, "multistream": 20,
+                      "cross_attn": 400, "sampler": 2000, "qkv": 50}[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -622,8 +809,8 @@ def main():
         run_reference(args, rank)
         return
     if args.workload != "step":
-        {"schedule": run_schedule, "cross_attn": run_cross_attn, "sampler": run_sampler,
-         "qkv": run_qkv}[args.workload](
+        {"schedule": run_schedule, "dense": run_dense, "multistream": run_multistream,
+         "cross_attn": run_cross_attn, "sampler": run_sampler, "qkv": run_qkv}[args.workload](
             args, rank, world, local)
         if world > 1:
             import torch.distributed as dist
