@@ -83,6 +83,26 @@ def test_prompt_batch_ragged_text(pv):
     assert torch.equal(got, want)
 
 
+def test_run_time_hand_out_is_repeatable(pv):
+    # short items are handed out at run time from a counter in the workspace
+    # (which CTA takes which item depends on timing); the last CTA returns the
+    # counter to zero, so repeated launches on one workspace give the same
+    # output bit for bit and leave the counters at zero
+    n_k = synth.text_lengths(8, seed=3)
+    n_q = [T] * 8
+    assert pv.pv_attn_plan(n_q, n_k, H)[1] == 1
+    qs, ks, vs, out, lse, ws = _run_varlen(pv, n_q, n_k)
+    q = torch.cat([p.reshape(-1) for p in qs])
+    k = torch.cat([p.reshape(-1) for p in ks])
+    v = torch.cat([p.reshape(-1) for p in vs])
+    out2 = torch.empty_like(out)
+    for _ in range(3):
+        pv.pv_attn_varlen(q, k, v, n_q, n_k, H, D, out2, None, ws, ws.numel())
+        torch.cuda.synchronize()
+        assert torch.equal(out, out2)
+        assert int(torch.count_nonzero(ws[:256 + 8])) == 0  # error word, both counters
+
+
 def test_small_head_dim_and_tails(pv):
     # D = 64, query and key counts that leave ragged 128-row tiles
     n_q, n_k = [1, 129, 300], [7, 130, 385]
