@@ -190,8 +190,8 @@ PV_API pv_status pv_qkv_ws_bytes(int tokens, int dim, size_t* ws_bytes);
  * of k, v into the per-step store exactly as pv_rope_append, q_rot likewise.
  *  x: bf16 [tokens][dim] (the listed streams' tokens back to back, in list
  *     order), w: bf16 [3 dim][dim] (W_q, W_k, W_v rows, a linear layer's
- *     [out][in]), bias: f32 [3 dim] (4-byte aligned), g_q, g_k: f32 [dim]
- *     (16-byte aligned), eps > 0.  Misaligned pointers: PV_ERR_INVALID_ARG.
+ *     [out][in]), bias: f32 [3 dim], g_q, g_k: f32 [dim] (all 16-byte
+ *     aligned), eps > 0.  Misaligned pointers: PV_ERR_INVALID_ARG.
  *  ws: device workspace of pv_qkv_ws_bytes, 256-byte aligned (holds y in
  *     f32 and the per-token sums of squares; no need to clear it).
  * Two launches: a tcgen05 GEMM whose epilogue adds the bias and sums the

@@ -664,9 +664,8 @@ pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int la
     if (!x || !w || !bias || !g_q || !g_k || !q_rot || !ws)
         return fail(PV_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned(x, 16) || !aligned(w, 16) || !aligned(q_rot, 16) || !aligned(ws, 256) ||
-        !aligned(bias, 4) || !aligned(g_q, 16) || !aligned(g_k, 16))
-        return fail(PV_ERR_INVALID_ARG,
-                    "x, w, q_rot, g_q, g_k 16-byte, ws 256-byte, bias 4-byte aligned");
+        !aligned(bias, 16) || !aligned(g_q, 16) || !aligned(g_k, 16))
+        return fail(PV_ERR_INVALID_ARG, "x, w, q_rot, bias, g_q, g_k 16-byte, ws 256-byte aligned");
     if (!(eps > 0.f) || !std::isfinite(eps)) return fail(PV_ERR_INVALID_ARG, "eps must be > 0");
     const pv_kv_config& c = kv->cfg;
     const int dim = c.heads * c.head_dim;

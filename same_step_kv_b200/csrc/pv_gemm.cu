@@ -16,9 +16,9 @@
 // 148 SMs).  Warp 0 loads 64-column slices of x and w with TMA into a ring
 // of stages (128-byte swizzle); warp 1 runs the issue loop with all lanes and
 // one elected lane issues the tcgen05.mma (M = 128, N = BN, K = 16, one f32
-// accumulator per half in TMEM); warps 4-7 (one TMEM lane quadrant each, one
-// token of each half per thread) add the bias, sum the squares and stage the
-// tile in the freed ring for TMA stores.  A half beyond the last token is
+// accumulator per half in TMEM); then all 8 warps (two per TMEM lane
+// quadrant, one per half, one token per thread) add the bias, sum the squares
+// and stage the tile in the freed ring for TMA stores.  A half beyond the last token is
 // neither loaded nor multiplied.  Every wait on an mbarrier is bounded.
 #include "pv_internal.h"
 
@@ -40,8 +40,9 @@ struct GCfg {
     static constexpr int kStages = BN == 256 ? 3 : kGMaxStages;
     static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr int kSmem = kBarOff + 256 + 1024;
-    // the epilogue stages 4 warps x 32 tokens x BN f32 (one half) in the freed ring
-    static_assert(4 * 32 * BN * 4 <= kBarOff, "epilogue staging does not fit the ring");
+    // the epilogue stages 8 warps x 32 tokens x kEpiCols f32 per round in the freed ring
+    static constexpr int kEpiCols = BN < 128 ? BN : 128;
+    static_assert(8 * 32 * kEpiCols * 4 <= kBarOff, "epilogue staging does not fit the ring");
     static_assert(kBarOff + 256 + 1024 <= 227 * 1024, "shared memory");
 };
 
@@ -238,38 +239,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
         while (!g_try(g_smem(&b->done), 0) && clock64() - t0 < kGWait) {
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // epilogue: one token of each half per thread, TMEM lane quadrant q4
-        const int q4 = warp - 4;
+    }
+    // epilogue, all 8 warps: warp w reads TMEM lane quadrant w % 4 (one token
+    // per thread) of half (w < 4 ? 1 : 0), so two warps share each SMSP
+    {
+        const int q4 = warp & 3;
+        const int u = warp < 4 ? 1 : 0;
         const bool ok = __all_sync(0xffffffffu, g_wait(g_smem(&b->done), 0, b, err));
-        if (ok && !*(volatile int*)&b->abort) {
+        if (ok && u < halves && !*(volatile int*)&b->abort) {
             g_fence_after();
             const int kind = n0 / dim;  // 0: q, 1: k, 2: v
-            // 32 tokens x BN f32 of this warp, in 32-column boxes of 4 KB,
+            constexpr int kCols = C::kEpiCols;  // columns staged per round
+            // 32 tokens x kCols f32 of this warp, in 32-column boxes of 4 KB,
             // staged in the ring that the MMAs no longer read
-            uint8_t* buf = smem + q4 * (32 * BN * 4);
-            for (int u = 0; u < halves; ++u) {
-                const int row0 = m0 + u * kGM + q4 * 32;  // this warp's first token
-                const int grow = row0 + lane;
-                if (u > 0) {
-                    // the previous half's stores have read the staging buffer
+            uint8_t* buf = smem + warp * (32 * kCols * 4);
+            const int row0 = m0 + u * kGM + q4 * 32;  // this warp's first token
+            const int grow = row0 + lane;
+            float sq = 0.f;
+            for (int c0 = 0; c0 < BN; c0 += kCols) {
+                if (c0 > 0) {
+                    // the previous round's stores have read the staging buffer
                     if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                     __syncwarp();
                 }
-                float sq = 0.f;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
+                for (int c = c0; c < c0 + kCols; c += 32) {
                     uint32_t o[32];
                     g_tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + u * BN + c, o);
-                    uint8_t* box = buf + (c / 32) * 4096;
+                    uint8_t* box = buf + ((c - c0) / 32) * 4096;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float* bj = bias + n0 + c + 4 * j;
+                        const float4 bj = __ldg(reinterpret_cast<const float4*>(bias + n0 + c + 4 * j));
                         float4 v;
-                        v.x = __uint_as_float(o[4 * j + 0]) + __ldg(bj + 0);
-                        v.y = __uint_as_float(o[4 * j + 1]) + __ldg(bj + 1);
-                        v.z = __uint_as_float(o[4 * j + 2]) + __ldg(bj + 2);
-                        v.w = __uint_as_float(o[4 * j + 3]) + __ldg(bj + 3);
+                        v.x = __uint_as_float(o[4 * j + 0]) + bj.x;
+                        v.y = __uint_as_float(o[4 * j + 1]) + bj.y;
+                        v.z = __uint_as_float(o[4 * j + 2]) + bj.z;
+                        v.w = __uint_as_float(o[4 * j + 3]) + bj.w;
                         sq = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, sq))));
                         // 16-byte chunk j of row `lane`, 128-byte swizzle
                         *reinterpret_cast<float4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
@@ -278,12 +283,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0 && row0 < tokens) {
-                    for (int c = 0; c < BN; c += 32)
-                        g_tma_store(&ty, g_smem(buf + (c / 32) * 4096), n0 + c, row0);
+                    for (int c = c0; c < c0 + kCols; c += 32)
+                        g_tma_store(&ty, g_smem(buf + ((c - c0) / 32) * 4096), n0 + c, row0);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
-                if (kind < 2 && grow < tokens) atomicAdd(ss + (size_t)grow * 2 + kind, sq);
             }
+            if (kind < 2 && grow < tokens) atomicAdd(ss + (size_t)grow * 2 + kind, sq);
             if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
             __syncwarp();
         }
