@@ -122,10 +122,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Bars* b
     return true;
 }
 
-#ifndef PV_MMA_SPIN
-#define PV_MMA_SPIN 1
-#endif
-
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -141,7 +137,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // Bounded wait that never suspends the thread: for the single MMA-issuing
 // thread, whose reaction time is on the critical path of every tile.
 __device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, Bars* b, int* err) {
-#if PV_MMA_SPIN
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
@@ -155,9 +150,6 @@ __device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, Bars* b
             }
         }
     }
-#else
-    return mbar_wait(bar, parity, b, err);
-#endif
 }
 
 // ----------------------------------------------------------------- TMA
@@ -578,9 +570,6 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     __syncwarp();
 }
 
-#ifndef PV_TRACK_MAX
-#define PV_TRACK_MAX 0
-#endif
 // Exponentials of 64 of this thread's scores: p = 2^(s*sl2 - m) on the XU
 // pipe, written to TMEM as bf16 pairs at tP (32 columns, one store; fewer,
 // larger stores than 16-column ones measured 4 % faster per launch).  The
