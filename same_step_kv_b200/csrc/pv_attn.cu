@@ -122,36 +122,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Bars* b
     return true;
 }
 
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait that never suspends the thread: for the single MMA-issuing
-// thread, whose reaction time is on the critical path of every tile.
-__device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, Bars* b, int* err) {
-    if (mbar_test(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 255) == 0) {
-            if (*(volatile int*)&b->abort) return false;
-            if (clock64() - t0 > kWaitCycles) {
-                atomicExch(err, 1);
-                *(volatile int*)&b->abort = 1;
-                return false;
-            }
-        }
-    }
-}
-
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
                                          uint32_t bar) {
@@ -468,8 +438,8 @@ template <int D, bool kRun>
 __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t tmem) {
     using C = Cfg<D>;
     // every lane waits; the vote reconverges the warp before the next issue
-    auto wspin = [&](uint32_t bar, uint32_t par, Bars* bb, int* err) -> bool {
-        const bool r = mbar_spin(bar, par, bb, err);
+    auto wwait = [&](uint32_t bar, uint32_t par, Bars* bb, int* err) -> bool {
+        const bool r = mbar_wait(bar, par, bb, err);
         return __all_sync(0xffffffffu, r);
     };
     constexpr uint32_t idesc_qk = idesc_bf16(kQRows, kKeyTile, false);
@@ -504,11 +474,11 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     // a segment overwrites O, which the previous segment's epilogue must
     // have read out first.
     auto do_pv = [&](int X, int stage, int j) -> bool {
-        if (j == 0 && !wspin(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
-        if (!wspin(smem_u32(&b->p_lo[X]), pc[X] & 1, b, p.err)) return false;
+        if (j == 0 && !wwait(smem_u32(&b->o_empty[X]), (oc[X] & 1) ^ 1, b, p.err)) return false;
+        if (!wwait(smem_u32(&b->p_lo[X]), pc[X] & 1, b, p.err)) return false;
         tc_fence_after();
         pv(X, stage, j > 0, 0);          // keys 0..63 while the softmax does 64..127
-        if (!wspin(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
+        if (!wwait(smem_u32(&b->p_full[X]), pc[X] & 1, b, p.err)) return false;
         ++pc[X];
         tc_fence_after();
         pv(X, stage, true, kKeyTile / 32);
@@ -519,7 +489,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
     Seg g;
     while (ok && (kRun ? item_take(p, b, rk, g, ok) : it.next(p, g))) {
         const bool hasB = g.rows[1] > 0;
-        if (!(ok = wspin(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
+        if (!(ok = wwait(smem_u32(&b->q_full), qseg & 1, b, p.err))) break;
         ++qseg;
         tc_fence_after();
         const int n = g.n;
@@ -529,11 +499,11 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
             const int vs_prev = (kv + 2 * j - 1) % C::kStages;
             const uint32_t vph_prev = ((kv + 2 * j - 1) / C::kStages) & 1;
             if (j > 0) {
-                if (!(ok = wspin(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
+                if (!(ok = wwait(smem_u32(&b->kv_full[vs_prev]), vph_prev, b, p.err) &&
                            do_pv(0, vs_prev, j - 1)))
                     break;
             }
-            if (!(ok = wspin(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
+            if (!(ok = wwait(smem_u32(&b->kv_full[ks]), kph, b, p.err))) break;
             tc_fence_after();
             qk(0, ks);
             tc_commit_e(smem_u32(&b->s_full[0]));
@@ -549,7 +519,7 @@ __device__ void mma_issuer(const AttnParams& p, uint8_t* smem, Bars* b, uint32_t
         tc_commit_e(smem_u32(&b->q_empty));  // the Q tiles are free once these S products end
         const int vs = (kv + 2 * n - 1) % C::kStages;
         const uint32_t vph = ((kv + 2 * n - 1) / C::kStages) & 1;
-        if (!(ok = wspin(smem_u32(&b->kv_full[vs]), vph, b, p.err) && do_pv(0, vs, n - 1)))
+        if (!(ok = wwait(smem_u32(&b->kv_full[vs]), vph, b, p.err) && do_pv(0, vs, n - 1)))
             break;
         tc_commit_e(smem_u32(&b->o_full[0]));
         ++oc[0];
