@@ -230,7 +230,8 @@ PV_API pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_di
  * are read from the next head (or as zeros past the buffer) and masked out,
  * so k and v must hold finite values.
  * ws: device workspace of pv_attn_dense_ws_bytes bytes, zero-filled by the
- * caller before its first use (the kernels leave it zeroed again). */
+ * caller before its first use (the kernels leave it zeroed again; after a
+ * call whose device wait gave up, zero it again). */
 PV_API pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, int n_k,
                         int heads, int head_dim, void* out, float* lse, void* ws,
                         size_t ws_bytes, void* cuda_stream);
@@ -255,7 +256,8 @@ PV_API pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* 
  *  out: bf16 [sum n_q][H][D], token-major, sequence i from token
  *    n_q[0] + ... + n_q[i-1].  lse: optional f32 [sum n_q][H].
  *  ws: device workspace of pv_attn_varlen_ws_bytes bytes, zero-filled before
- *    its first use, 256-byte aligned. */
+ *    its first use (and again after a call whose device wait gave up),
+ *    256-byte aligned. */
 PV_API pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs,
                                 const int* n_q, const int* n_k, int heads, int head_dim,
                                 void* out, float* lse, void* ws, size_t ws_bytes,
@@ -326,18 +328,20 @@ PV_API pv_status pv_euler_cfg_step(float* x, const float* v_cond, const float* v
 PV_API pv_status pv_x0_estimate(float* x0, const float* x, const float* v, size_t n,
                                 float sigma, void* cuda_stream);
 
-/* Self-test of the attention kernel's software exponential: y[i] = 2^x[i]
- * computed as that kernel computes a quarter of its softmax exponentials
- * (round-to-nearest range reduction and a fitted minimax cubic; maximum
- * relative error 7.5e-5 for x in [-125, 128)).  x, y: f32 device arrays of n
- * elements.  Used by the tests to compare against exp2. */
+/* Self-test of a software exponential on the FMA pipe: y[i] = 2^x[i] by
+ * round-to-nearest range reduction and a fitted minimax cubic (maximum
+ * relative error 7.5e-5 for x in [-125, 128)).  Moving a share of the
+ * softmax exponentials onto it measured slower at every share, so the
+ * attention kernel computes them all with ex2; the function is kept tested
+ * for hardware where the balance of the pipes differs.  x, y: f32 device
+ * arrays of n elements.  Used by the tests to compare against exp2. */
 PV_API pv_status pv_selftest_exp2_poly(const float* x, float* y, size_t n, void* cuda_stream);
 
 /* Reads (synchronously) and clears the device error word that the kernels of
  * this handle set when a bounded device-side wait gives up.  *code is 0 when
  * no wait timed out; otherwise the call returns PV_ERR_TIMEOUT and also
- * re-zeroes the workspace's split-merge arrival counters, which an aborted
- * launch may have left part counted. */
+ * re-zeroes the workspace's counters (split-merge arrivals, run-time item
+ * hand-out), which an aborted launch may have left part counted. */
 PV_API pv_status pv_kv_poll_device_error(pv_kv kv, int* code);
 
 /* Failure-path self-test: launches one device-side wait on a barrier that
