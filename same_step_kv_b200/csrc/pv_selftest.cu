@@ -1,4 +1,4 @@
-// Self-test entry point: the attention kernel's polynomial exp2, elementwise.
+// Self-test entry point: the polynomial exp2 of pv_math.cuh, elementwise.
 #include "pv_internal.h"
 #include "pv_math.cuh"
 
