@@ -154,22 +154,28 @@ def test_dense_video_18480(pv):
     store.close()
 
 
-def test_dense_score_spikes_force_rescale(pv):
+@pytest.mark.parametrize("n_q", [256, 100, 300])
+def test_dense_score_spikes_force_rescale(pv, n_q):
     """A later key tile whose scores exceed the running maximum by far more
     than the lazy-rescale threshold (log2 units): the running maximum moves
-    and O and l are rescaled inside a segment.  Half the heads get such spikes: keys of 5.0 against queries near 2.0 lift
-    the score by ~112 over the first tile's maximum, ~161 in log2 units, and
-    a key of 10.0 further on lifts it by as much again.  Without the rescale
-    those exponentials overflow to inf.  The spikes sit in tiles that are not
+    and O and l are rescaled inside a segment.  Half the heads get such
+    spikes: keys of 5.0 against queries near 2.0 lift the score by ~112 over
+    the first tile's maximum, ~161 in log2 units, and a key of 10.0 further
+    on lifts it by as much again.  Without the rescale those exponentials
+    overflow to inf.  The spikes sit in odd and even key tiles that are not
     the first of their segment (24 heads x 32 key tiles over 148 SMs:
-    stream-K segments of ~5 tiles)."""
-    n_q, n_k, heads, dim = 256, 4096, 24, 128
+    stream-K segments of ~5 tiles).  256 queries: two query tiles per
+    segment; 100: one (S of the next key tile computed ahead, in the other S
+    buffer, and O rescaled after the previous P V has completed); 300: both
+    kinds in one launch (a 44-row last query block)."""
+    n_k, heads, dim = 4096, 24, 128
     g = torch.Generator().manual_seed(5)
     q = (2.0 + 0.01 * torch.randn(heads, n_q, dim, generator=g)).to(torch.bfloat16)
     k = (0.3 * torch.randn(heads, n_k, dim, generator=g)).to(torch.bfloat16)
     v = torch.randn(heads, n_k, dim, generator=g).to(torch.bfloat16)
     q[heads // 2:] = torch.randn(heads - heads // 2, n_q, dim, generator=g).to(torch.bfloat16)
-    for pos in (3 * 128 + 5, 9 * 128 + 77, 17 * 128, 25 * 128 + 127, 30 * 128 + 40):
+    for pos in (1 * 128 + 3, 3 * 128 + 5, 9 * 128 + 77, 17 * 128, 22 * 128 + 64, 25 * 128 + 127,
+                30 * 128 + 40):
         k[: heads // 2, pos] = 5.0
     k[: heads // 2, 31 * 128 + 9] = 10.0
     q, k, v = q.cuda(), k.cuda(), v.cuda()

@@ -103,6 +103,36 @@ def test_run_time_hand_out_is_repeatable(pv):
         assert int(torch.count_nonzero(ws[:256 + 8])) == 0  # error word, both counters
 
 
+def test_run_time_one_tile_items_rescale(pv):
+    # 64 sequences of 100 queries (one query tile per item) against 512 keys:
+    # 1,536 items of 4 key tiles, handed out at run time.  In half the heads
+    # keys of 5.0 and 10.0 in key tiles 1, 2 and 3 move the running maximum
+    # far past the lazy-rescale threshold, so O is rescaled after the P V of
+    # the previous key tile, with S of the next one already computed
+    n, nq, nk, heads = 64, 100, 512, 8
+    assert pv.pv_attn_plan([nq] * n, [nk] * n, heads)[1] == 1
+    g = torch.Generator().manual_seed(11)
+    q = (2.0 + 0.01 * torch.randn(n, heads, nq, D, generator=g)).to(torch.bfloat16)
+    k = (0.3 * torch.randn(n, heads, nk, D, generator=g)).to(torch.bfloat16)
+    v = torch.randn(n, heads, nk, D, generator=g).to(torch.bfloat16)
+    for pos, val in ((128 + 3, 5.0), (2 * 128 + 100, 5.0), (3 * 128 + 9, 10.0)):
+        k[:, : heads // 2, pos] = val
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty(n * nq, heads, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(n * nq, heads, dtype=torch.float32, device="cuda")
+    wsb = pv.pv_attn_varlen_ws_bytes([nq] * n, [nk] * n, heads, D)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_attn_varlen(q, k, v, [nq] * n, [nk] * n, heads, D, out, lse, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(torch.count_nonzero(ws[:256 + 8])) == 0  # no wait gave up; counters reset
+    for i in (0, 17, 63):
+        for h in (0, 3, 4, 7):
+            rows = slice(i * nq, (i + 1) * nq)
+            o_ref, lse_ref = attention.attend(f64(q[i, h]), f64(k[i, h]), f64(v[i, h]))
+            assert_attn_close(f64(out[rows, h]), o_ref, f"seq {i} head {h}")
+            assert_lse_close(f64(lse[rows, h]), lse_ref, f"seq {i} head {h}")
+
+
 def test_small_head_dim_and_tails(pv):
     # D = 64, query and key counts that leave ragged 128-row tiles
     n_q, n_k = [1, 129, 300], [7, 130, 385]
