@@ -11,7 +11,7 @@ every layer is pre-filled, and the working set (6.9 GB of K/V) is far larger
 than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload step|cross_attn|sampler|qkv]
+                    [--workload step|schedule|dense|multistream|cross_attn|sampler|qkv]
 
 Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 on the host cores on a bounded sample of the same workload.
@@ -780,7 +780,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 100 for step, 400 for cross_attn, 2000 for sampler)")
+                    help="timed steps (default: step 100, schedule 3, dense 20, multistream 20, "
+                         "cross_attn 400, sampler 2000, qkv 50)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
