@@ -39,6 +39,7 @@ LATENT = 48 * 44 * 80           # values of one latent frame
 ATTN_FLOPS = 4 * T * N_KEYS * HEADS * D          # one chunk_attn launch
 ROPE_BYTES = 6 * T * HEADS * D * 2               # q,k,v read; q_rot,k_rot,v written
 WORKLOAD = "steady chunk 880 q x 18480 k, 24x128, 30 layers + Euler 48x44x80"
+METRIC = "chunk-attention TFLOP/s (whole step: 30 x rope_append + chunk_attn, Euler)"
 
 
 def load_peaks():
@@ -170,7 +171,7 @@ def run_reference(args, rank):
             vals.append(fl / dt / 1e12)
     v = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": "chunk-attention TFLOP/s", "value": v,
+        "impl": "reference", "metric": METRIC, "value": v,
         "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "higher_is_better": True, "scaling": "weak", "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD,
@@ -945,7 +946,7 @@ def main():
         achieved = ATTN_FLOPS / (attn_ms * 1e-3) / 1e12
         peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
         line = {
-            "metric": "chunk-attention TFLOP/s (whole step: 30 x rope_append + chunk_attn, Euler)",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
