@@ -136,19 +136,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-def oracle_sample(heads=HEADS):
-    """The fp64 oracle on one layer of the workload: RoPE of the chunk's q and k
-    and the attention of all 880 queries of `heads` heads over 18,480 keys.
-    Returns (flops, seconds, threads)."""
-    import numpy as np
-    import torch
-    from oracle import attention, rope
+def oracle_inputs(heads=HEADS):
+    """Host fp64 inputs of one layer of the workload for the first `heads`
+    heads: the chunk's q, k, v and the pre-filled K/V history.  The history
+    is drawn for those heads only; it is head-major, so that draw is exactly
+    the first `heads` heads of the full one."""
     from same_step_kv_b200 import synth
     q, k, v = synth.chunk_qkv(0, CHUNK, STEP, 0, T, HEADS, D)
-    kf, vf = synth.store_fill(0, 0, STEP, HEADS, N_KEYS, D)
+    kf, vf = synth.store_fill(0, 0, STEP, heads, N_KEYS, D)
     q, k, v = (t[:, :heads].double().numpy() for t in (q, k, v))
-    K = kf[:heads].double().numpy().transpose(1, 0, 2).copy()
-    V = vf[:heads].double().numpy().transpose(1, 0, 2).copy()
+    K = kf.double().numpy().transpose(1, 0, 2).copy()
+    V = vf.double().numpy().transpose(1, 0, 2).copy()
+    return q, k, v, K, V
+
+
+def oracle_sample(inputs):
+    """The fp64 oracle on one layer of the workload: RoPE of the chunk's q and
+    k, their append into the ring slot, and the attention of all 880 queries
+    of the inputs' heads over 18,480 keys.  Returns (flops, seconds, threads).
+    The append writes the same rows every time, so samples repeat exactly."""
+    import torch
+    from oracle import attention, rope
+    q, k, v, K, V = inputs
+    heads = q.shape[1]
     t0 = time.perf_counter()
     f, hh, ww = rope.token_coords(T, W, HH, 2 + CHUNK)
     qr = rope.rotate(q, f, hh, ww)
@@ -165,8 +175,9 @@ def run_reference(args, rank):
     if rank != 0:
         return
     vals = []
+    inputs = oracle_inputs(heads=2)
     for i in range(args.warmup + args.steps):
-        fl, dt, thr = oracle_sample(heads=2)
+        fl, dt, thr = oracle_sample(inputs)
         if i >= args.warmup:
             vals.append(fl / dt / 1e12)
     v = statistics.median(vals)
@@ -933,7 +944,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        runs = [oracle_sample() for _ in range(4)]
+        inputs = oracle_inputs()
+        runs = [oracle_sample(inputs) for _ in range(4)]
         fl, dt = runs[0][0], statistics.median(r[1] for r in runs)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": runs[0][2], "kind": "oracle",
                "sample": "one of the 30 layers of a step (RoPE + 880 x 18480 attention, "

@@ -11,10 +11,15 @@ import bench
 def _run(monkeypatch, capsys, rank):
     calls = []
 
-    def fake_sample(heads=bench.HEADS):
-        calls.append(heads)
-        return bench.ATTN_FLOPS * heads // bench.HEADS, 2.0, 7
+    def fake_inputs(heads=bench.HEADS):
+        calls.append(("inputs", heads))
+        return heads
 
+    def fake_sample(inputs):
+        calls.append(("sample", inputs))
+        return bench.ATTN_FLOPS * inputs // bench.HEADS, 2.0, 7
+
+    monkeypatch.setattr(bench, "oracle_inputs", fake_inputs)
     monkeypatch.setattr(bench, "oracle_sample", fake_sample)
     args = types.SimpleNamespace(gpus=1, steps=2, warmup=3)
     bench.run_reference(args, rank)
@@ -23,7 +28,8 @@ def _run(monkeypatch, capsys, rank):
 
 def test_reference_line_matches_the_gpu_arm(monkeypatch, capsys):
     calls, lines = _run(monkeypatch, capsys, rank=0)
-    assert len(calls) == 5 and len(lines) == 1          # warm-up + timed samples, one line
+    # inputs drawn once, then warm-up + timed samples of 2 heads; one line
+    assert calls == [("inputs", 2)] + [("sample", 2)] * 5 and len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference"
     assert d["metric"] == bench.METRIC
