@@ -76,7 +76,8 @@ typedef struct pv_kv_config {
     int heads;         /* H */
     int head_dim;      /* D: 64 or 128 */
     int frame_w;       /* tokens per row of a latent frame (40 at 1280 px) */
-    int frame_h;       /* token rows of a latent frame (22 at 704 px) */
+    int frame_h;       /* token rows of a latent frame (22 at 704 px);
+                          frame_w * frame_h <= 2^24 */
     int first_frames;  /* F0: latent frames of the first chunk (3) */
     int ring_slots;    /* R: recent chunks kept besides the sink (18), 1..PV_MAX_RING */
     int steps;         /* denoising steps per chunk (4) */
@@ -84,7 +85,7 @@ typedef struct pv_kv_config {
     int rope_pairs_t;  /* RoPE pairs of the time axis   (22 for D = 128, 12 for D = 64) */
     int rope_pairs_h;  /* RoPE pairs of the height axis (21 for D = 128, 10 for D = 64) */
     int rope_pairs_w;  /* RoPE pairs of the width axis  (21 for D = 128, 10 for D = 64) */
-    int max_frames;    /* largest latent-frame index + 1 that RoPE may see */
+    int max_frames;    /* largest latent-frame index + 1 that RoPE may see, <= 2^20 */
     double rope_theta; /* RoPE base (10000) */
 } pv_kv_config;
 
@@ -226,9 +227,10 @@ PV_API pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_di
 
 /* Plain softmax attention on explicit head-major buffers, the same kernel as
  * pv_chunk_attn:  q [H][n_q][D], k and v [H][n_k][D] bf16, out [n_q][H][D]
- * bf16, lse optional f32 [n_q][H].  Key rows past n_k inside a 128-key tile
- * are read from the next head (or as zeros past the buffer) and masked out,
- * so k and v must hold finite values.
+ * bf16, lse optional f32 [n_q][H].  1 <= n_q, n_k <= 2^30 and H * n_q,
+ * H * n_k < 2^31 (rows of one tensor map), else PV_ERR_SHAPE.  Key rows
+ * past n_k inside a 128-key tile are read from the next head (or as zeros
+ * past the buffer) and masked out, so k and v must hold finite values.
  * ws: device workspace of pv_attn_dense_ws_bytes bytes, zero-filled by the
  * caller before its first use (the kernels leave it zeroed again; after a
  * call whose device wait gave up, zero it again). */
@@ -247,7 +249,8 @@ PV_API pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* 
  * to the prompt's real length; chapter 4: the context holds no sequence
  * positions, so no RoPE, and no mask), one sequence per prompt.
  *  n_q, n_k: HOST arrays of n_seqs lengths (1 <= n_seqs <= PV_MAX_STREAMS);
- *    n_q[i] = 0 skips sequence i; n_q[i] > 0 needs n_k[i] >= 1.
+ *    n_q[i] = 0 skips sequence i; n_q[i] > 0 needs n_k[i] >= 1; every length
+ *    <= 2^30 and H * sum n_q, H * sum n_k < 2^31, else PV_ERR_SHAPE.
  *  q: the sequences' head-major blocks back to back, bf16: block i is
  *    [H][n_q[i]][D] and starts at row H * (n_q[0] + ... + n_q[i-1]).
  *  k, v: likewise [H][n_k[i]][D] blocks.  Rows past a block's last key inside

@@ -61,6 +61,10 @@ struct WsLayout {
     int n_counters, n_partials, n_table;
 };
 
+constexpr int kMaxLen = 1 << 30;          // queries or keys of one sequence at most
+constexpr int kMaxFrameTokens = 1 << 24;  // tokens of one latent frame at most
+constexpr int kMaxFramesCfg = 1 << 20;    // RoPE table rows of the time axis at most
+
 int tokens_per_frame(const pv_kv_config& c) { return c.frame_w * c.frame_h; }
 
 WsLayout ws_layout(const pv_kv_config& c) {
@@ -102,6 +106,13 @@ pv_status check_config(const pv_kv_config* c) {
                     c->rope_pairs_t, c->rope_pairs_h, c->rope_pairs_w, c->head_dim / 2);
     if (!(c->rope_theta > 1.0) || !std::isfinite(c->rope_theta))
         return fail(PV_ERR_SHAPE, "rope_theta must be finite and > 1");
+    // bounds before any int product of these fields (tokens per frame, the
+    // RoPE table's rows) is formed
+    if ((long long)c->frame_w * c->frame_h > kMaxFrameTokens)
+        return fail(PV_ERR_SHAPE, "frame of %d x %d tokens above %d", c->frame_w, c->frame_h,
+                    kMaxFrameTokens);
+    if (c->max_frames > kMaxFramesCfg)
+        return fail(PV_ERR_SHAPE, "max_frames %d above %d", c->max_frames, kMaxFramesCfg);
     const int T = tokens_per_frame(*c);
     const long long ltot = (long long)(c->first_frames + c->ring_slots) * T;
     const long long rows = (long long)c->layers * c->steps * c->max_streams * c->heads * ltot;
@@ -333,6 +344,9 @@ pv_status varlen_sizes(int n_seqs, const int* n_q, const int* n_k, int heads, in
         if (n_q[i] < 0 || n_k[i] < 0 || (n_q[i] > 0 && n_k[i] == 0))
             return fail(PV_ERR_SHAPE, "sequence %d: n_q %d, n_k %d (queries need keys)", i, n_q[i],
                         n_k[i]);
+        if (n_q[i] > kMaxLen || n_k[i] > kMaxLen)
+            return fail(PV_ERR_SHAPE, "sequence %d: n_q %d, n_k %d above %d", i, n_q[i], n_k[i],
+                        kMaxLen);
         const size_t qb = (n_q[i] + kQBlock - 1) / kQBlock;
         *n_cnt += (size_t)heads * qb * kQTilesPerCta;
         *tiles += (size_t)heads * qb * ((n_k[i] + kKeyTile - 1) / kKeyTile);
@@ -773,7 +787,7 @@ pv_status pv_rope_dense(pv_kv kv, int n_tokens, int frame0, const void* q, const
     const pv_kv_config& c = kv->cfg;
     if (n_tokens < 1 || n_tokens % kv->T != 0)
         return fail(PV_ERR_SHAPE, "n_tokens %d is not a positive multiple of %d", n_tokens, kv->T);
-    if (frame0 < 0 || frame0 + n_tokens / kv->T > c.max_frames)
+    if (frame0 < 0 || (long long)frame0 + n_tokens / kv->T > c.max_frames)
         return fail(PV_ERR_SHAPE, "frames %d..%d outside the RoPE table (max_frames %d)", frame0,
                     frame0 + n_tokens / kv->T - 1, c.max_frames);
     if ((long long)n_tokens * c.heads >= (1LL << 31))
@@ -818,6 +832,8 @@ pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_dim, size
     if (!ws_bytes) return fail(PV_ERR_INVALID_ARG, "output pointer is NULL");
     if (n_q < 1 || n_k < 1 || heads < 1 || (head_dim != 64 && head_dim != 128))
         return fail(PV_ERR_SHAPE, "bad dense attention shape");
+    if (n_q > kMaxLen || n_k > kMaxLen)
+        return fail(PV_ERR_SHAPE, "n_q %d or n_k %d above %d", n_q, n_k, kMaxLen);
     const size_t n_qb = (n_q + kQBlock - 1) / kQBlock;
     const size_t n_cnt = (size_t)heads * n_qb * kQTilesPerCta;
     const size_t tiles = (size_t)heads * n_qb * ((n_k + kKeyTile - 1) / kKeyTile);
@@ -833,6 +849,8 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
     if (!q || !k || !v || !out) return fail(PV_ERR_INVALID_ARG, "NULL tensor pointer");
     if (n_q < 1 || n_k < 1 || heads < 1 || (head_dim != 64 && head_dim != 128))
         return fail(PV_ERR_SHAPE, "n_q, n_k, heads must be positive and head_dim 64 or 128");
+    if (n_q > kMaxLen || n_k > kMaxLen)
+        return fail(PV_ERR_SHAPE, "n_q %d or n_k %d above %d", n_q, n_k, kMaxLen);
     if ((long long)n_q * heads >= (1LL << 31) || (long long)n_k * heads >= (1LL << 31))
         return fail(PV_ERR_SHAPE, "too many rows for a tensor map");
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))

@@ -70,6 +70,8 @@ extern "C" pv_status pv_attn_dense_noalloc(const void* q, const void* k, const v
     if (n_q < 1 || n_k < 1 || heads < 1 || (head_dim != 64 && head_dim != 128))
         return report_error(PV_ERR_SHAPE, "pv_attn_dense_noalloc: n_q, n_k, heads must be "
                                           "positive and head_dim 64 or 128");
+    if (n_q > (1 << 30) || n_k > (1 << 30))  // the rounded tile counts stay in int
+        return report_error(PV_ERR_SHAPE, "pv_attn_dense_noalloc: n_q or n_k above 2^30");
     if ((long long)n_q * heads >= (1LL << 31) || (long long)n_k * heads >= (1LL << 31))
         return report_error(PV_ERR_SHAPE, "pv_attn_dense_noalloc: too many rows for a tensor map");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))

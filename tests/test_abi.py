@@ -122,7 +122,10 @@ def test_max_frames_bounds_the_schedule():
 
 @pytest.mark.parametrize("bad", [
     dict(head_dim=96), dict(ring_slots=0), dict(ring_slots=65), dict(steps=9),
-    dict(rope_pairs=(10, 10, 10)), dict(max_streams=65), dict(rope_theta=1.0)])
+    dict(rope_pairs=(10, 10, 10)), dict(max_streams=65), dict(rope_theta=1.0),
+    # sizes whose int products would overflow: rejected before they are formed
+    dict(frame_w=65536, frame_h=65536), dict(frame_w=4097, frame_h=4096),
+    dict(max_frames=(1 << 20) + 1), dict(max_frames=(1 << 31) - 1)])
 def test_bad_configs_are_rejected(bad):
     kw = dict(layers=1, heads=2, head_dim=64, frame_w=8, frame_h=4)
     kw.update({k: v for k, v in bad.items() if k in kw})
@@ -226,6 +229,27 @@ def test_varlen_workspace_and_shape_checks():
         assert e.value.status == pv.PV_ERR_SHAPE
     # no queries anywhere: a no-op that touches no device
     pv.pv_attn_varlen(0, 0, 0, [0, 0], [3, 0], 2, 64, 0, None, 0, 0)
+
+
+def test_lengths_above_two_to_the_30_are_rejected():
+    # a length near 2^31 would overflow the int tile counts (n + 255) / 256;
+    # every entry point rejects lengths above 2^30 before forming them
+    big, ok = (1 << 30) + 1, 1 << 30
+    assert pv.pv_attn_dense_ws_bytes(ok, 1, 1, 64) > 0
+    calls = [
+        lambda: pv.pv_attn_dense_ws_bytes(big, 1, 1, 64),
+        lambda: pv.pv_attn_dense_ws_bytes(1, (1 << 31) - 1, 1, 64),
+        lambda: pv.pv_attn_varlen_ws_bytes([big], [1], 1, 64),
+        lambda: pv.pv_attn_varlen_ws_bytes([1], [(1 << 31) - 1], 1, 64),
+        lambda: pv.pv_attn_plan([(1 << 31) - 1], [1], 1),
+        # pointers are checked for NULL only before the shapes, never touched
+        lambda: pv.pv_attn_dense(256, 256, 256, (1 << 31) - 1, 1, 1, 64, 256, None, 256, 0),
+        lambda: pv.pv_attn_dense_noalloc(256, 256, 256, 1, big, 1, 64, 256),
+    ]
+    for call in calls:
+        with pytest.raises(pv.PVError) as e:
+            call()
+        assert e.value.status == pv.PV_ERR_SHAPE
 
 
 # ------------------------------------------------------------------ q/k/v projection (host checks)
