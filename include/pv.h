@@ -24,12 +24,13 @@
  *    A fault of an earlier asynchronous launch surfaces as PV_ERR_CUDA on a
  *    later call.  pv_last_error() gives a one-line message for the calling
  *    thread's most recent failure.
- *  - Workspaces: attention launches keep split-KV partial results and
- *    arrival counters in their workspace (a handle's for pv_chunk_attn, the
- *    `ws` argument for pv_attn_dense, pv_attn_varlen and
- *    pv_qkv_rope_append).  Launches that use one workspace must not overlap
- *    on the GPU: issue them on one CUDA stream, or order them with events.
- *    The host side of a handle is guarded by a mutex.
+ *  - Workspaces hold a launch's scratch state: split-KV partial results and
+ *    arrival counters for attention (a handle's workspace for pv_chunk_attn,
+ *    the `ws` argument for pv_attn_dense and pv_attn_varlen), the projected
+ *    q/k/v and their sums of squares for pv_qkv_rope_append.  Launches that
+ *    use one workspace must not overlap on the GPU: issue them on one CUDA
+ *    stream, or order them with events.  The host side of a handle is
+ *    guarded by a mutex.
  *  - Element types: "bf16" is IEEE bfloat16 (2 bytes), "f32" is float.
  *  - Device pointers must be 16-byte aligned; the KV store must be 256-byte
  *    aligned.
