@@ -239,8 +239,11 @@ PV_API pv_status pv_attn_dense_ws_bytes(int n_q, int n_k, int heads, int head_di
  * past n_k inside a 128-key tile are read from the next head (or as zeros
  * past the buffer) and masked out, so k and v must hold finite values.
  * ws: device workspace of pv_attn_dense_ws_bytes bytes, zero-filled by the
- * caller before its first use (the kernels leave it zeroed again; after a
- * call whose device wait gave up, zero it again). */
+ * caller before its first use (the kernels leave it zeroed again).  Its first
+ * int is the device error word: nonzero after a call whose bounded device
+ * wait gave up (that call's out / lse are then incomplete).
+ * pv_attn_poll_device_error reads it and, if set, zeroes the workspace
+ * again. */
 PV_API pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, int n_k,
                         int heads, int head_dim, void* out, float* lse, void* ws,
                         size_t ws_bytes, void* cuda_stream);
@@ -266,8 +269,8 @@ PV_API pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* 
  *  out: bf16 [sum n_q][H][D], token-major, sequence i from token
  *    n_q[0] + ... + n_q[i-1].  lse: optional f32 [sum n_q][H].
  *  ws: device workspace of pv_attn_varlen_ws_bytes bytes, zero-filled before
- *    its first use (and again after a call whose device wait gave up),
- *    256-byte aligned. */
+ *    its first use, 256-byte aligned.  Its first int is the device error
+ *    word, as for pv_attn_dense (pv_attn_poll_device_error). */
 PV_API pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs,
                                 const int* n_q, const int* n_k, int heads, int head_dim,
                                 void* out, float* lse, void* ws, size_t ws_bytes,
@@ -304,7 +307,11 @@ PV_API pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int he
  *    before any stream capture.
  *  - Every call shares the one array and clears the part it needs on
  *    cuda_stream; calls whose executions overlap on the GPU (other streams,
- *    other host threads) race on it and must be serialised by the caller. */
+ *    other host threads) race on it and must be serialised by the caller.
+ *  - A bounded device wait that gives up (about one second) leaves out / lse
+ *    incomplete and sets the array's device error word, which the next call
+ *    clears: read it after the call with pv_attn_poll_device_error(NULL, 0,
+ *    ...) on the same stream. */
 PV_API pv_status pv_attn_dense_noalloc(const void* q, const void* k, const void* v, int n_q,
                                        int n_k, int heads, int head_dim, void* out, float* lse,
                                        void* cuda_stream);
@@ -338,21 +345,30 @@ PV_API pv_status pv_euler_cfg_step(float* x, const float* v_cond, const float* v
 PV_API pv_status pv_x0_estimate(float* x0, const float* x, const float* v, size_t n,
                                 float sigma, void* cuda_stream);
 
-/* Self-test of a software exponential on the FMA pipe: y[i] = 2^x[i] by
- * round-to-nearest range reduction and a fitted minimax cubic (maximum
- * relative error 7.5e-5 for x in [-125, 128)).  Moving a share of the
- * softmax exponentials onto it measured slower at every share, so the
- * attention kernel computes them all with ex2; the function is kept tested
- * for hardware where the balance of the pipes differs.  x, y: f32 device
- * arrays of n elements.  Used by the tests to compare against exp2. */
-PV_API pv_status pv_selftest_exp2_poly(const float* x, float* y, size_t n, void* cuda_stream);
-
 /* Reads (synchronously) and clears the device error word that the kernels of
  * this handle set when a bounded device-side wait gives up.  *code is 0 when
  * no wait timed out; otherwise the call returns PV_ERR_TIMEOUT and also
  * re-zeroes the workspace's counters (split-merge arrivals, run-time item
  * hand-out), which an aborted launch may have left part counted. */
 PV_API pv_status pv_kv_poll_device_error(pv_kv kv, int* code);
+
+/* Reads and clears the device error word of an attention workspace: ws and
+ * ws_bytes as given to pv_attn_dense or pv_attn_varlen, or ws = NULL for the
+ * fixed scratch of pv_attn_dense_noalloc (ws_bytes ignored).  Waits for
+ * cuda_stream first (synchronous).  *code is 0 when no device wait gave up;
+ * otherwise the call zeroes the workspace (the scratch's error word only,
+ * since each no-alloc call clears its counters itself) and returns
+ * PV_ERR_TIMEOUT: the output of the call that timed out is incomplete.
+ * A ws that is not 256-byte aligned or under 256 bytes: PV_ERR_INVALID_ARG. */
+PV_API pv_status pv_attn_poll_device_error(void* ws, size_t ws_bytes, int* code,
+                                           void* cuda_stream);
+
+/* Failure-path self-test of the workspace entry points: one device-side wait
+ * on a barrier that nothing arrives on gives up after about one second and
+ * records a timeout in the error word of ws (NULL: the no-alloc scratch),
+ * exactly as a wait of the attention kernel would; the context stays usable.
+ * Asynchronous on cuda_stream. */
+PV_API pv_status pv_attn_selftest_wait_timeout(void* ws, void* cuda_stream);
 
 /* Failure-path self-test: launches one device-side wait on a barrier that
  * nothing ever arrives on.  Like every wait of the attention kernel it gives

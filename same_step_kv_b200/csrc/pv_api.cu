@@ -1081,6 +1081,57 @@ pv_status pv_kv_poll_device_error(pv_kv kv, int* code) {
     return PV_OK;
 }
 
+// The device error word of an attention workspace (ws), or of the fixed
+// scratch of pv_attn_dense_noalloc (ws == NULL), and the bytes to re-zero
+// after a timeout: the whole workspace (its arrival counters may be left part
+// counted), or only the scratch's error block (each no-alloc call clears the
+// counters it uses).
+static pv_status attn_err_word(void* ws, size_t ws_bytes, char** base, size_t* clear) {
+    if (ws) {
+        if (!aligned(ws, 256) || ws_bytes < 256)
+            return fail(PV_ERR_INVALID_ARG, "workspace %p of %zu bytes: need >= 256, 256-byte aligned",
+                        ws, ws_bytes);
+        *base = (char*)ws;
+        *clear = ws_bytes;
+        return PV_OK;
+    }
+    void* p = nullptr;
+    cudaError_t e = noalloc_scratch_address(&p);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the no-alloc scratch");
+    *base = (char*)p;
+    *clear = 256;
+    return PV_OK;
+}
+
+pv_status pv_attn_poll_device_error(void* ws, size_t ws_bytes, int* code, void* cuda_stream) {
+    if (!code) return fail(PV_ERR_INVALID_ARG, "NULL argument");
+    *code = 0;
+    char* base = nullptr;
+    size_t clear = 0;
+    pv_status st = attn_err_word(ws, ws_bytes, &base, &clear);
+    if (st) return st;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)cuda_stream);
+    if (e == cudaSuccess) e = cudaMemcpy(code, base, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (*code) {
+        e = cudaMemset(base, 0, clear);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+        return fail(PV_ERR_TIMEOUT, "a device-side wait gave up (code %d)", *code);
+    }
+    return PV_OK;
+}
+
+pv_status pv_attn_selftest_wait_timeout(void* ws, void* cuda_stream) {
+    char* base = nullptr;
+    size_t clear = 0;
+    pv_status st = attn_err_word(ws, ws ? 256 : 0, &base, &clear);
+    if (st) return st;
+    if ((st = check_async("an earlier launch"))) return st;
+    cudaError_t e = launch_wait_timeout_probe((int*)base, (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait-timeout self-test launch");
+    return PV_OK;
+}
+
 pv_status pv_kv_selftest_wait_timeout(pv_kv kv, void* cuda_stream) {
     if (!kv) return fail(PV_ERR_INVALID_ARG, "handle is NULL");
     if (!kv->device) return fail(PV_ERR_STATE, "bookkeeping-only handle has no device buffers");

@@ -151,6 +151,10 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// GPU-scope acquire-release fence: this thread's earlier global writes are
+// visible to any thread that later synchronises with it at GPU scope (the
+// split-KV arrival count), and the other way round for later reads.
+__device__ __forceinline__ void fence_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 // Make this thread's shared-memory writes visible to the async (TMA) proxy.
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -634,8 +638,9 @@ __device__ __forceinline__ void stage_flush(const CUtensorMap* to, const uint8_t
 // the partial slot of CTA c_first + k; with `keep` this CTA's own part is
 // still in TMEM (tO, m_own, l_own) and is taken from there, bit for bit the
 // values it stored.  Sums run in part order whichever CTA merges, so results
-// are reproducible.  The (m, l) loads are issued four parts at a time and a
-// part's 32-column block in one batch: a merge costs a few L2 round trips.
+// are reproducible.  The (m, l) loads are issued four parts at a time (one
+// pass) and a part's 32-column block in one batch: a merge costs a few L2
+// round trips.
 template <int D>
 __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, int X, int r,
                                             bool row_ok, bool keep, uint32_t tO, float m_own,
@@ -647,28 +652,25 @@ __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, i
     auto ml = [&](int k) -> const float* {
         return p.partial + part_slot(p, g.c_first + k, g.i0, X) * slot_f + (size_t)kQRows * D;
     };
-    float M = -INFINITY;
-    for (int k0 = 0; k0 < g.nseg; k0 += 4) {
-        float mk[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u;
-            mk[u] = k == self ? m_own : (k < g.nseg ? __ldcg(ml(k) + r) : -INFINITY);
-        }
-        M = fmaxf(fmaxf(M, fmaxf(mk[0], mk[1])), fmaxf(mk[2], mk[3]));
-    }
-    float L = 0.f;
+    // running (M, L) over the parts in order, L relative to M: one batch of
+    // loads per four parts
+    float M = -INFINITY, L = 0.f;
     for (int k0 = 0; k0 < g.nseg; k0 += 4) {
         float mk[4], lk[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int k = k0 + u;
-            mk[u] = k == self ? m_own : (k < g.nseg ? __ldcg(ml(k) + r) : 0.f);
+            mk[u] = k == self ? m_own : (k < g.nseg ? __ldcg(ml(k) + r) : -INFINITY);
             lk[u] = k == self ? l_own : (k < g.nseg ? __ldcg(ml(k) + kQRows + r) : 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (k0 + u < g.nseg) L += lk[u] * ex2(mk[u] - M);
+        for (int u = 0; u < 4; ++u) {
+            if (k0 + u < g.nseg) {
+                const float Mn = fmaxf(M, mk[u]);
+                L = L * ex2(M - Mn) + lk[u] * ex2(mk[u] - Mn);
+                M = Mn;
+            }
+        }
     }
     const float invL = 1.0f / L;
 #pragma unroll 1
@@ -837,7 +839,7 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
         // all four warps' partial rows are visible before the arrival count
         // moves; bounded waits on mbarriers, not bar.sync, so that an
         // aborting CTA can never block here
-        __threadfence();
+        fence_gpu();
         __syncwarp();
         if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&b->ep_in[X]));
         if (r == 0) {
@@ -855,7 +857,7 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&b->ep_out[X]), ec & 1, b, p.err));
         ++ec;
         if (ok && b->last[X]) {
-            __threadfence();
+            fence_gpu();
             merge_parts<D>(p, g, X, r, row_ok, keep, tO, m, l, dst,
                            p.lse ? p.lse + (size_t)tok * p.heads + g.head : nullptr, to, ebuf,
                            warp_full, tok_w);
@@ -953,13 +955,9 @@ template <int D, bool kRun>
 cudaError_t launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& to, const AttnParams& p, cudaStream_t s) {
     using C = Cfg<D>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kRun>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(attn_kernel<D, kRun>, C::kSmem, configured);
+    if (e != cudaSuccess) return e;
     attn_kernel<D, kRun><<<p.grid, kThreads, C::kSmem, s>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }

@@ -308,13 +308,9 @@ cudaError_t launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const C
                            const float* bias, float* ss, int tokens, int dim, int* err,
                            cudaStream_t s) {
     using C = GCfg<BN>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(qkv_gemm_kernel<BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<unsigned long long> configured{0};
+    const cudaError_t e = smem_limit_once(qkv_gemm_kernel<BN>, C::kSmem, configured);
+    if (e != cudaSuccess) return e;
     dim3 grid((tokens + kGM * kGHalves - 1) / (kGM * kGHalves), 3 * dim / BN);
     qkv_gemm_kernel<BN><<<grid, kGThreads, C::kSmem, s>>>(tx, tw, ty, bias, ss, tokens, dim, err);
     return cudaGetLastError();

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "../../include/pv.h"
 
@@ -127,6 +128,27 @@ bool encode_out_map(CUtensorMap* map, void* out, long long tokens, int heads, in
                     size_t errlen);
 bool encode_rows_map(CUtensorMap* map, const void* base, long long rows, int D, char* err,
                      size_t errlen);
+
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to a device, so it is set once per device:
+// `done` holds one bit per device ordinal below 64 (others set it on every
+// call).  Two host threads that race here both set the same value.
+template <typename K>
+cudaError_t smem_limit_once(K kernel, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (bit) done.fetch_or(bit, std::memory_order_release);
+    return cudaSuccess;
+}
+
+// Device address, on the current device, of the fixed scratch array of
+// pv_attn_dense_noalloc (its first 256 bytes hold the device error word).
+cudaError_t noalloc_scratch_address(void** out);
 
 // Records a failure for pv_last_error() and returns code.
 pv_status report_error(pv_status code, const char* msg);

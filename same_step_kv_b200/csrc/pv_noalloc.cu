@@ -57,6 +57,9 @@ cudaError_t scratch_address(void** out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
+
+cudaError_t noalloc_scratch_address(void** out) { return scratch_address(out); }
+
 }  // namespace pv
 
 using namespace pv;

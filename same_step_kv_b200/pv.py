@@ -78,8 +78,9 @@ _SIGS = {
     "pv_attn_dense_noalloc": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp], _i),
     "pv_euler_step": ([_vp, _vp, _sz, ctypes.c_float, _vp], _i),
     "pv_kv_poll_device_error": ([_vp, ctypes.POINTER(_i)], _i),
-    "pv_selftest_exp2_poly": ([_vp, _vp, _sz, _vp], _i),
     "pv_kv_selftest_wait_timeout": ([_vp, _vp], _i),
+    "pv_attn_poll_device_error": ([_vp, _sz, ctypes.POINTER(_i), _vp], _i),
+    "pv_attn_selftest_wait_timeout": ([_vp, _vp], _i),
     "pv_attn_varlen_ws_bytes": ([_i, _vp, _vp, _i, _i, ctypes.POINTER(_sz)], _i),
     "pv_attn_varlen": ([_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _vp, _vp, _vp, _sz, _vp], _i),
     "pv_attn_plan": ([_i, _vp, _vp, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
@@ -309,8 +310,16 @@ def pv_kv_selftest_wait_timeout(kv, cuda_stream=None) -> None:
     _check(lib.pv_kv_selftest_wait_timeout(kv, _stream(cuda_stream)))
 
 
-def pv_selftest_exp2_poly(x, y, n, cuda_stream=None) -> None:
-    _check(lib.pv_selftest_exp2_poly(_ptr(x), _ptr(y), n, _stream(cuda_stream)))
+def pv_attn_poll_device_error(ws=None, ws_bytes=0, cuda_stream=None) -> int:
+    """ws=None: the fixed scratch of pv_attn_dense_noalloc."""
+    c = _i()
+    _check(lib.pv_attn_poll_device_error(_ptr(ws), ws_bytes, ctypes.byref(c),
+                                         _stream(cuda_stream)))
+    return c.value
+
+
+def pv_attn_selftest_wait_timeout(ws=None, cuda_stream=None) -> None:
+    _check(lib.pv_attn_selftest_wait_timeout(_ptr(ws), _stream(cuda_stream)))
 
 
 # ------------------------------------------------------------------ helpers
