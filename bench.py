@@ -480,7 +480,8 @@ SAMPLER_FRAMES = 248   # 8 streams x 31 latent frames
 def run_sampler(args, rank, world, local):
     """One sampler step over a batch of SAMPLER_FRAMES latent frames (48 x 44 x 80
     each): the CFG-guided Euler update (x, v_cond, v_uncond in, x out: 16 B per
-    value) and the x0 estimate (x, v in, x0 out: 12 B per value)."""
+    value), the plain Euler update of a second latent batch (x, v in, x out:
+    12 B per value) and the x0 estimate (x, v in, x0 out: 12 B per value)."""
     import torch
     from same_step_kv_b200 import pv, synth
     torch.cuda.set_device(local)
@@ -495,6 +496,7 @@ def run_sampler(args, rank, world, local):
     vc = synth.normal_f32(synth.seed_of(0x5A02, rank), (n,), dev)
     vu = synth.normal_f32(synth.seed_of(0x5A03, rank), (n,), dev)
     x0 = torch.empty_like(x)
+    xe = synth.normal_f32(synth.seed_of(0x5A04, rank), (n,), dev)
     sig = pv.pv_sigma_schedule(40, 12.0)[0]
     d = float(sig[21] - sig[20])
     w = 5.0
@@ -509,11 +511,12 @@ def run_sampler(args, rank, world, local):
         if record:
             e1.record(cs)
             ev.append((e0, e1))
+        pv.pv_euler_step(xe, vu, n, d, cs)
         pv.pv_x0_estimate(x0, x, vc, n, float(sig[21]), cs)
 
     ms_step, clocks = timed_steps(step, args, local, world, cs)
     cfg_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    step_bytes = 16 * n + 12 * n
+    step_bytes = 16 * n + 12 * n + 12 * n
     # e2e: velocities in from pinned host memory, x0 read back
     hvc, hvu = vc.cpu().pin_memory(), vu.cpu().pin_memory()
     hx0 = torch.empty(n, dtype=torch.float32).pin_memory()
@@ -522,6 +525,7 @@ def run_sampler(args, rank, world, local):
         vc.copy_(hvc, non_blocking=True)
         vu.copy_(hvu, non_blocking=True)
         pv.pv_euler_cfg_step(x, vc, vu, n, w, d, cs)
+        pv.pv_euler_step(xe, vu, n, d, cs)
         pv.pv_x0_estimate(x0, x, vc, n, float(sig[21]), cs)
         hx0.copy_(x0, non_blocking=True)
 
@@ -531,7 +535,7 @@ def run_sampler(args, rank, world, local):
         hbm = float(peaks["hbm_gbs"])
         a = 16 * n / (cfg_ms * 1e-3) / 1e9
         line = {
-            "metric": "sampler GB/s (CFG-guided Euler step + x0 estimate)",
+            "metric": "sampler GB/s (CFG-guided Euler step, Euler step, x0 estimate)",
             "value": step_bytes * world / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -544,7 +548,7 @@ def run_sampler(args, rank, world, local):
                          "ms_per_launch": cfg_ms, "traffic": None},
             "e2e": {"value": step_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": 8 * n, "d2h_bytes_per_step": 4 * n},
-            "gpu_launches": 2 * args.steps, "clocks": clocks, "cpu_baseline": None,
+            "gpu_launches": 3 * args.steps, "clocks": clocks, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
 

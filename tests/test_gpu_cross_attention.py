@@ -167,3 +167,25 @@ def test_varlen_rejects_bad_arguments(pv):
     assert e.value.status == pv.PV_ERR_CAPACITY
     # no queries at all: nothing to do
     pv.pv_attn_varlen(x, x, x, [0, 0], [3, 0], 2, 64, x, None, ws, ws.numel())
+
+
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_ragged_one_tile_blocks_stream_k_every_row(pv, head_dim):
+    # ragged sequences whose last query block holds a single tile (112, 100,
+    # 44 and 1 rows over a multiple of 256) beside ones whose blocks all hold
+    # two (1024, 129 queries), cut stream-K into split parts that the last CTA
+    # to arrive merges; every row of every head
+    n_q = [880, 100, 1024, 300, 129, 1]
+    n_k = [3000, 2500, 1200, 4100, 700, 3333]
+    heads = 3
+    assert pv.pv_attn_plan(n_q, n_k, heads)[1] == 0   # stream-K
+    qs, ks, vs, out, lse, ws = _run_varlen(pv, n_q, n_k, heads, head_dim)
+    _check(qs, ks, vs, out, lse, n_q, range(heads))
+    assert int(ws[:256].view(torch.int32)[0]) == 0
+    # the arrival counters are back at zero: a second launch is bit-identical
+    out2 = torch.empty_like(out)
+    pv.pv_attn_varlen(torch.cat([t.reshape(-1) for t in qs]), torch.cat([t.reshape(-1) for t in ks]),
+                      torch.cat([t.reshape(-1) for t in vs]), n_q, n_k, heads, head_dim, out2, None,
+                      ws, ws.numel())
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)

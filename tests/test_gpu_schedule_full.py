@@ -5,7 +5,11 @@ its 4 steps, the sigma = 0 sink pass, then 28 one-frame chunks of 4 steps
 the oracle session follows layer 1 for two of the heads through every call
 (RoPE, append, ring) and checks sampled query rows at sampled calls, so the
 bookkeeping of all 117 calls and the key sets up to 18,480 keys are
-compared against the plain definition."""
+compared against the plain definition.  The checked calls cover every phase
+and every edge of the ring's fill: the first chunk's first and last steps,
+the sink pass, chunks 1 and 2 (one and two ring slots), 17 and 18 (the ring
+filling), 19 and 20 (the first wraps) and 28 (the last chunk); the rows sit
+at query-tile edges and in the one-tile last block of each frame."""
 import numpy as np
 import pytest
 import torch
@@ -20,9 +24,10 @@ pytestmark = pytest.mark.gpu
 W, HH, H, D, R, L = 40, 22, 24, 128, 18, 2
 T = W * HH
 LAYER = 1                      # the layer the oracle follows
-HEADS = [0, 17]                # the heads the oracle follows
-ROWS = [0, 39, 440, 879]       # query rows checked (of each 880-token frame)
-CHECK = {(0, 3), (0, "sink"), (1, 0), (17, 2), (18, 1), (19, 3), (28, 2)}
+HEADS = [0, 9, 17, 23]         # the heads the oracle follows
+ROWS = [0, 39, 127, 128, 440, 767, 768, 879]   # query rows checked (of each 880-token frame)
+CHECK = {(0, 0), (0, 3), (0, "sink"), (1, 0), (2, 1), (17, 2), (18, 1), (18, 3), (19, 3),
+         (20, 0), (28, 2), (28, 3)}
 
 
 @pytest.fixture(scope="module")
