@@ -24,129 +24,102 @@ __device__ __forceinline__ uint32_t pack(float lo, float hi) {
 // Blog "Learning Video Generation from the Wan2.2 Source Code", chapter 4,
 // "3D RoPE": pair p of a head belongs to the time, height or width block and
 // turns by that coordinate times the pair's frequency, as the complex product
-// (x + i y) e^{i angle}.  An item is 8 consecutive dimensions (4 pairs) of one
-// (token, head) of q, k and v; rows are read and written with 128-bit
-// coalesced accesses.  The grid is one resident wave and each thread takes
-// its items two at a time, both items' loads issued before either is used,
-// so that enough bytes are in flight to cover the memory latency.
+// (x + i y) e^{i angle}.  One thread handles 8 consecutive dimensions (4
+// pairs) of one (token, head) of q, k and v; rows are read and written with
+// 128-bit coalesced accesses.
 // kProj = false: q, k, v are bf16 [tokens][H][D].
 // kProj = true: they are the f32 projection y [tokens][3 * dim] (pv_gemm.cu)
 // and q, k get the rest of the QK-Norm first (same chapter): times
 // rsqrt(ss / dim + eps), ss the token's sum of squares, then the gain.
-struct RopeItem {
-    float qf[8], kf[8];
-    uint4 vv;
-    int t, h, g;
-};
-
-template <bool kProj>
-__device__ __forceinline__ void rope_load(const RopeParams& p, const RopeStreamDesc& sd, int it,
-                                          int per_tok, int G, RopeItem& x) {
-    x.t = it / per_tok;
-    const int j = it - x.t * per_tok;
-    x.h = j / G;
-    x.g = j - x.h * G;
-    if (kProj) {
-        const int dim = p.heads * p.head_dim;
-        const int f0 = x.h * p.head_dim + x.g * 8;           // feature of this group
-        const size_t row = (size_t)(sd.in_tok0 + x.t);
-        const float* yq = p.y + row * 3 * dim + f0;
-        const float sq = rsqrtf(__ldg(p.ss + row * 2) / dim + p.eps);
-        const float sk = rsqrtf(__ldg(p.ss + row * 2 + 1) / dim + p.eps);
-        const float4 q0 = __ldcs(reinterpret_cast<const float4*>(yq));
-        const float4 q1 = __ldcs(reinterpret_cast<const float4*>(yq + 4));
-        const float4 k0 = __ldcs(reinterpret_cast<const float4*>(yq + dim));
-        const float4 k1 = __ldcs(reinterpret_cast<const float4*>(yq + dim + 4));
-        const float4 v0 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim));
-        const float4 v1 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim + 4));
-        // the gains as four 16-byte loads (f0 is a multiple of 8)
-        const float4 gq0 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0));
-        const float4 gq1 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0 + 4));
-        const float4 gk0 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0));
-        const float4 gk1 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0 + 4));
-        const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-        const float gqa[8] = {gq0.x, gq0.y, gq0.z, gq0.w, gq1.x, gq1.y, gq1.z, gq1.w};
-        const float gka[8] = {gk0.x, gk0.y, gk0.z, gk0.w, gk1.x, gk1.y, gk1.z, gk1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            x.qf[i] = qa[i] * sq * gqa[i];
-            x.kf[i] = ka[i] * sk * gka[i];
-        }
-        x.vv = make_uint4(pack(v0.x, v0.y), pack(v0.z, v0.w), pack(v1.x, v1.y), pack(v1.z, v1.w));
-    } else {
-        const size_t in_off = ((size_t)(sd.in_tok0 + x.t) * p.heads + x.h) * p.head_dim + x.g * 8;
-        const uint4 qv = ld_stream(p.q + in_off);
-        const uint4 kv = ld_stream(p.k + in_off);
-        x.vv = ld_stream(p.v + in_off);
-        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float2 a = unpack(qw[u]);
-            const float2 b = unpack(kw[u]);
-            x.qf[2 * u] = a.x;
-            x.qf[2 * u + 1] = a.y;
-            x.kf[2 * u] = b.x;
-            x.kf[2 * u + 1] = b.y;
-        }
-    }
-}
-
-__device__ __forceinline__ void rope_store(const RopeParams& p, const RopeStreamDesc& sd,
-                                           const RopeItem& x) {
-    const int T = p.frame_w * p.frame_h;
-    const int f = sd.frame0 + x.t / T;
-    const int r = x.t % T;
-    const int hh = r / p.frame_w;
-    const int ww = r - hh * p.frame_w;
-    uint32_t qo[4], ko[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int pair = x.g * 4 + u;
-        int idx;
-        if (pair < p.pairs_t) {
-            idx = f * p.pairs_t + pair;
-        } else if (pair < p.pairs_t + p.pairs_h) {
-            idx = p.tab_h0 + hh * p.pairs_h + (pair - p.pairs_t);
-        } else {
-            idx = p.tab_w0 + ww * p.pairs_w + (pair - p.pairs_t - p.pairs_h);
-        }
-        const float2 cs = __ldg(p.table + idx);
-        const float ax = x.qf[2 * u], ay = x.qf[2 * u + 1];
-        const float bx = x.kf[2 * u], by = x.kf[2 * u + 1];
-        qo[u] = pack(fmaf(ax, cs.x, -ay * cs.y), fmaf(ax, cs.y, ay * cs.x));
-        ko[u] = pack(fmaf(bx, cs.x, -by * cs.y), fmaf(bx, cs.y, by * cs.x));
-    }
-    const size_t qrow = (size_t)sd.qrot_row0 + (size_t)x.h * sd.n_tok + x.t;
-    st16(p.q_rot + qrow * p.head_dim + x.g * 8, make_uint4(qo[0], qo[1], qo[2], qo[3]));
-    const uint4 kout = make_uint4(ko[0], ko[1], ko[2], ko[3]);
-    for (int d = 0; d < sd.n_dst; ++d) {
-        const size_t row = (size_t)sd.dst_row0[d] + (size_t)x.h * p.dst_head_stride + x.t;
-        st16(p.k_dst + row * p.head_dim + x.g * 8, kout);
-        st16(p.v_dst + row * p.head_dim + x.g * 8, x.vv);
-    }
-}
-
 template <bool kProj>
 __global__ void __launch_bounds__(256) rope_append_kernel(const __grid_constant__ RopeParams p) {
     const RopeStreamDesc& sd = p.st[blockIdx.y];
     const int G = p.head_dim >> 3;                   // 16-byte groups per head row
     const int per_tok = p.heads * G;
     const int n_items = sd.n_tok * per_tok;
-    const int stride = gridDim.x * blockDim.x;
-    int it = blockIdx.x * blockDim.x + threadIdx.x;
-    for (; it + stride < n_items; it += 2 * stride) {
-        RopeItem a, b;
-        rope_load<kProj>(p, sd, it, per_tok, G, a);
-        rope_load<kProj>(p, sd, it + stride, per_tok, G, b);
-        rope_store(p, sd, a);
-        rope_store(p, sd, b);
-    }
-    if (it < n_items) {
-        RopeItem a;
-        rope_load<kProj>(p, sd, it, per_tok, G, a);
-        rope_store(p, sd, a);
+    const int T = p.frame_w * p.frame_h;
+    for (int it = blockIdx.x * blockDim.x + threadIdx.x; it < n_items; it += gridDim.x * blockDim.x) {
+        const int t = it / per_tok;
+        const int j = it - t * per_tok;
+        const int h = j / G;
+        const int g = j - h * G;
+        float qf[8], kf[8];
+        uint4 vv;
+        if (kProj) {
+            const int dim = p.heads * p.head_dim;
+            const int f0 = h * p.head_dim + g * 8;           // feature of this group
+            const size_t row = (size_t)(sd.in_tok0 + t);
+            const float* yq = p.y + row * 3 * dim + f0;
+            const float sq = rsqrtf(__ldg(p.ss + row * 2) / dim + p.eps);
+            const float sk = rsqrtf(__ldg(p.ss + row * 2 + 1) / dim + p.eps);
+            const float4 q0 = __ldcs(reinterpret_cast<const float4*>(yq));
+            const float4 q1 = __ldcs(reinterpret_cast<const float4*>(yq + 4));
+            const float4 k0 = __ldcs(reinterpret_cast<const float4*>(yq + dim));
+            const float4 k1 = __ldcs(reinterpret_cast<const float4*>(yq + dim + 4));
+            const float4 v0 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim));
+            const float4 v1 = __ldcs(reinterpret_cast<const float4*>(yq + 2 * dim + 4));
+            // the gains as four 16-byte loads (f0 is a multiple of 8)
+            const float4 gq0 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0));
+            const float4 gq1 = __ldg(reinterpret_cast<const float4*>(p.g_q + f0 + 4));
+            const float4 gk0 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0));
+            const float4 gk1 = __ldg(reinterpret_cast<const float4*>(p.g_k + f0 + 4));
+            const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            const float gqa[8] = {gq0.x, gq0.y, gq0.z, gq0.w, gq1.x, gq1.y, gq1.z, gq1.w};
+            const float gka[8] = {gk0.x, gk0.y, gk0.z, gk0.w, gk1.x, gk1.y, gk1.z, gk1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                qf[i] = qa[i] * sq * gqa[i];
+                kf[i] = ka[i] * sk * gka[i];
+            }
+            vv = make_uint4(pack(v0.x, v0.y), pack(v0.z, v0.w), pack(v1.x, v1.y), pack(v1.z, v1.w));
+        } else {
+            const size_t in_off = ((size_t)(sd.in_tok0 + t) * p.heads + h) * p.head_dim + g * 8;
+            const uint4 qv = ld_stream(p.q + in_off);
+            const uint4 kv = ld_stream(p.k + in_off);
+            vv = ld_stream(p.v + in_off);
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 a = unpack(qw[u]);
+                const float2 b = unpack(kw[u]);
+                qf[2 * u] = a.x;
+                qf[2 * u + 1] = a.y;
+                kf[2 * u] = b.x;
+                kf[2 * u + 1] = b.y;
+            }
+        }
+        const int f = sd.frame0 + t / T;
+        const int r = t % T;
+        const int hh = r / p.frame_w;
+        const int ww = r - hh * p.frame_w;
+        uint32_t qo[4], ko[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int pair = g * 4 + u;
+            int idx;
+            if (pair < p.pairs_t) {
+                idx = f * p.pairs_t + pair;
+            } else if (pair < p.pairs_t + p.pairs_h) {
+                idx = p.tab_h0 + hh * p.pairs_h + (pair - p.pairs_t);
+            } else {
+                idx = p.tab_w0 + ww * p.pairs_w + (pair - p.pairs_t - p.pairs_h);
+            }
+            const float2 cs = __ldg(p.table + idx);
+            const float ax = qf[2 * u], ay = qf[2 * u + 1];
+            const float bx = kf[2 * u], by = kf[2 * u + 1];
+            qo[u] = pack(fmaf(ax, cs.x, -ay * cs.y), fmaf(ax, cs.y, ay * cs.x));
+            ko[u] = pack(fmaf(bx, cs.x, -by * cs.y), fmaf(bx, cs.y, by * cs.x));
+        }
+        const size_t qrow = (size_t)sd.qrot_row0 + (size_t)h * sd.n_tok + t;
+        st16(p.q_rot + qrow * p.head_dim + g * 8, make_uint4(qo[0], qo[1], qo[2], qo[3]));
+        const uint4 kout = make_uint4(ko[0], ko[1], ko[2], ko[3]);
+        for (int d = 0; d < sd.n_dst; ++d) {
+            const size_t row = (size_t)sd.dst_row0[d] + (size_t)h * p.dst_head_stride + t;
+            st16(p.k_dst + row * p.head_dim + g * 8, kout);
+            st16(p.v_dst + row * p.head_dim + g * 8, vv);
+        }
     }
 }
 
@@ -251,32 +224,12 @@ int sm_count() {
 
 }  // namespace
 
-// CTAs of `kernel` (256 threads) resident on one SM of the current device,
-// looked up once per device ordinal below 64.
-template <typename K>
-int resident_ctas(K kernel, std::atomic<int>* cache) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    if (dev >= 0 && dev < 64) {
-        const int c = cache[dev].load(std::memory_order_relaxed);
-        if (c > 0) return c;
-    }
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n <= 0)
-        n = 4;
-    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
-    return n;
-}
-
 cudaError_t launch_rope(const RopeParams& p, int max_tok, cudaStream_t s) {
     const long long items = (long long)max_tok * p.heads * (p.head_dim / 8);
     if (items >= (1LL << 31)) return cudaErrorInvalidValue;
-    static std::atomic<int> occ_plain[64] = {}, occ_proj[64] = {};
-    const int per_sm = p.y ? resident_ctas(rope_append_kernel<true>, occ_proj)
-                           : resident_ctas(rope_append_kernel<false>, occ_plain);
-    // grid: one resident wave shared by the streams, at most two items per thread
-    const int per_stream = (int)std::max<long long>(
-        1, std::min<long long>((items + 511) / 512, (long long)per_sm * sm_count() / p.n_streams));
+    // grid: enough CTAs per stream to cover the SMs a few times over
+    const int per_stream = (int)std::min<long long>((items + 255) / 256,
+                                                    std::max(1, 8 * sm_count() / p.n_streams));
     dim3 grid(per_stream, p.n_streams);
     if (p.y)
         rope_append_kernel<true><<<grid, 256, 0, s>>>(p);
