@@ -123,7 +123,8 @@ PV_API pv_status pv_last_error(char* buf, size_t len);
  *  kv_bytes: the KV store, 2 * layers * steps * max_streams * H * Ltot * D
  *            bf16 (K region followed by V region).
  *  ws_bytes: the workspace: RoPE cos/sin table, split-KV partial results,
- *            arrival counters and a device error word. */
+ *            arrival counters, the fused projection's flags and a device
+ *            error word. */
 PV_API pv_status pv_kv_required_bytes(const pv_kv_config* cfg, size_t* kv_bytes, size_t* ws_bytes);
 
 /* Creates a handle over caller buffers.  Checks cfg (D in {64,128}, RoPE
@@ -202,8 +203,19 @@ PV_API pv_status pv_qkv_ws_bytes(int tokens, int dim, size_t* ws_bytes);
  *     aligned), eps > 0.  Misaligned pointers: PV_ERR_INVALID_ARG.
  *  ws: device workspace of pv_qkv_ws_bytes, 256-byte aligned (holds y in
  *     f32 and the per-token sums of squares; no need to clear it).
- * Two launches: a tcgen05 GEMM whose epilogue adds the bias and sums the
- * squares, then the RoPE / append kernel, which applies the norm. */
+ * When every tile of the GEMM can be resident at once (tokens <= 1024 at
+ * dim 3072: the steady chunk) and the RoPE table fits in shared memory
+ * beside a tile, one cooperative launch: a tcgen05 GEMM whose epilogue adds
+ * the bias, writes each token's sum of squares over its tile, raises its
+ * flag in the handle's workspace, waits (bounded, about a second; a wait
+ * that gives up sets the handle's device error word) until every tile of
+ * the token's q or k has done so, adds their sums in tile order, then
+ * applies the norm, the gain and the rotation to the accumulator and writes
+ * bf16 q_rot and the K/V rows; y is not written.  Otherwise a memset and
+ * two launches: the GEMM writes y and adds the sums of squares, and the
+ * RoPE / append kernel applies the norm as it reads y.  Both round each
+ * output once to bf16.  The handle's workspace is used either way: calls
+ * on one handle must not overlap on the GPU. */
 PV_API pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int layer,
                                     int step, const void* x, const void* w, const float* bias,
                                     const float* g_q, const float* g_k, float eps, void* q_rot,

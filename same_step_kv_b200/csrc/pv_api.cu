@@ -55,9 +55,10 @@ struct StreamState {
     StreamState() { std::fill(slot_frame, slot_frame + PV_MAX_RING, -1); }
 };
 
-// Workspace layout: [error word | counters | RoPE table | partial slots].
+// Workspace layout: [error word | counters | projection flags | RoPE table |
+// partial slots].
 struct WsLayout {
-    size_t err_off, cnt_off, tab_off, part_off, total;
+    size_t err_off, cnt_off, flag_off, tab_off, part_off, total;
     int n_counters, n_partials, n_table;
 };
 
@@ -79,7 +80,8 @@ WsLayout ws_layout(const pv_kv_config& c) {
                 c.frame_w * c.rope_pairs_w;
     w.err_off = 0;
     w.cnt_off = 256;
-    w.tab_off = round_up(w.cnt_off + sizeof(int) * (size_t)w.n_counters, 256);
+    w.flag_off = round_up(w.cnt_off + sizeof(int) * (size_t)w.n_counters, 256);
+    w.tab_off = round_up(w.flag_off + sizeof(unsigned) * (size_t)kQkvFlags, 256);
     w.part_off = round_up(w.tab_off + sizeof(float2) * (size_t)w.n_table, 256);
     w.total = round_up(w.part_off + sizeof(float) * partial_slot_floats(c.head_dim) *
                                         (size_t)w.n_partials, 256);
@@ -242,6 +244,11 @@ struct pv_kv_s {
     char* ws = nullptr;
     WsLayout wl{};
     CUtensorMap tm_k{}, tm_v{};
+    // the K and V regions with 32-row boxes (stores of the fused projection)
+    CUtensorMap tm_k32{}, tm_v32{};
+    bool maps32 = false;
+    // the last call number of the fused projection (its flags' value)
+    unsigned qkv_epoch = 0;
     std::vector<StreamState> streams;
     std::mutex mu;
     // cached tensor map of the last q_rot buffer
@@ -449,6 +456,12 @@ pv_status pv_kv_init(pv_kv* out, const pv_kv_config* cfg, void* kv_dev, size_t k
             delete kv;
             return fail(PV_ERR_CUDA, "%s", msg);
         }
+        // without them pv_qkv_rope_append takes its two-launch path
+        kv->maps32 = region_rows(kv) < (1LL << 31) &&
+                     encode_2d_map(&kv->tm_k32, kv->kbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                   c.head_dim, region_rows(kv), 64, 32, msg, sizeof msg) &&
+                     encode_2d_map(&kv->tm_v32, kv->vbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                   c.head_dim, region_rows(kv), 64, 32, msg, sizeof msg);
     }
     *out = kv;
     return PV_OK;
@@ -632,8 +645,14 @@ pv_status rope_params(pv_kv kv, int n_streams, const int* streams, int layer, in
 }
 
 // Workspace of pv_qkv_rope_append: y f32 [tokens][3 * dim], then the sums of
-// squares f32 [tokens][2], each 256-byte aligned.
+// squares f32 [tokens][2][dim / tile width] (the fused launch writes one
+// partial sum per feature tile; the two-launch path adds into [tokens][2]),
+// each part 256-byte aligned.
 size_t qkv_y_bytes(long long tokens, int dim) { return round_up((size_t)tokens * 3 * dim * 4, 256); }
+size_t qkv_ss_bytes(long long tokens, int dim) {
+    const int bn = qkv_gemm_tile_n(dim);
+    return round_up((size_t)tokens * 2 * (bn ? dim / bn : 1) * 4, 256);
+}
 }  // namespace
 
 extern "C" {
@@ -665,7 +684,7 @@ pv_status pv_qkv_ws_bytes(int tokens, int dim, size_t* ws_bytes) {
     if (!ws_bytes) return fail(PV_ERR_INVALID_ARG, "output pointer is NULL");
     if (tokens < 1 || dim < 64 || dim % 64 != 0)
         return fail(PV_ERR_SHAPE, "tokens must be positive and dim a multiple of 64");
-    *ws_bytes = qkv_y_bytes(tokens, dim) + round_up((size_t)tokens * 2 * 4, 256);
+    *ws_bytes = qkv_y_bytes(tokens, dim) + qkv_ss_bytes(tokens, dim);
     return PV_OK;
 }
 
@@ -708,16 +727,40 @@ pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int la
                        sizeof msg))
         return fail(PV_ERR_CUDA, "%s", msg);
     cudaStream_t s = (cudaStream_t)cuda_stream;
-    cudaError_t e = cudaMemsetAsync(ss, 0, (size_t)tok * 2 * 4, s);
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the sums of squares");
-    e = launch_qkv_gemm(tx, tw, ty, bias, ss, tok, dim, (int*)(kv->ws + kv->wl.err_off), s);
-    if (e != cudaSuccess) return cuda_fail(e, "qkv projection launch");
+    int* err = (int*)(kv->ws + kv->wl.err_off);
+    cudaError_t e;
     p.y = y;
     p.ss = ss;
     p.g_q = g_q;
     p.g_k = g_k;
     p.eps = eps;
     p.q_rot = (bf16*)q_rot;
+    // one launch when every tile of the GEMM can be resident at once (the
+    // steady chunk's 880 tokens: 144 CTAs) and the rows fit TMA's 32-bit
+    // coordinates; else the GEMM writes y and the RoPE / append kernel
+    // reads it back
+    const long long qrows = (long long)c.heads * tok;
+    QkvOutMaps om;
+    if (kv->maps32 && qrows < (1LL << 31) &&
+        encode_2d_map(&om.q, q_rot, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c.head_dim, qrows, 64, 32,
+                      msg, sizeof msg)) {
+        om.k = kv->tm_k32;
+        om.v = kv->tm_v32;
+        // a new value for the flags of this call (0 is the cleared state)
+        unsigned epoch = kv->qkv_epoch + 1;
+        if (epoch == 0) epoch = 1;
+        unsigned* flags = (unsigned*)(kv->ws + kv->wl.flag_off);
+        e = launch_qkv_fused(tx, tw, bias, ss, flags, epoch, tok, dim, err, p, om, s);
+        if (e == cudaSuccess) {
+            kv->qkv_epoch = epoch;
+            return PV_OK;
+        }
+        if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail(e, "qkv fused launch");
+    }
+    e = cudaMemsetAsync(ss, 0, (size_t)tok * 2 * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the sums of squares");
+    e = launch_qkv_gemm(tx, tw, ty, bias, ss, tok, dim, err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "qkv projection launch");
     e = launch_rope(p, max_tok, s);
     if (e != cudaSuccess) return cuda_fail(e, "qkv rope_append launch");
     return PV_OK;

@@ -112,6 +112,25 @@ int qkv_gemm_tile_n(int dim);
 cudaError_t launch_qkv_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ty,
                             const float* bias, float* ss, int tokens, int dim, int* err,
                             cudaStream_t s);
+// Destinations of the fused epilogue's TMA stores, each [rows][head_dim]
+// bf16 with boxes of 32 rows x 64 features (128-byte swizzle): q_rot, the K
+// region and the V region.
+struct QkvOutMaps {
+    CUtensorMap q, k, v;
+};
+// The same GEMM with the QK-Norm, RoPE and append in its epilogue (one
+// cooperative launch).  ss [tokens][2][dim / tile width] takes one partial
+// sum of squares per feature tile (no need to clear it); CTA c sets
+// flags[c] = epoch once its partial sums are written, and the CTAs of a
+// token block read them once all of its tiles' flags hold epoch (flags of
+// earlier calls hold other values).  cudaErrorCooperativeLaunchTooLarge when
+// its tiles cannot all be resident, there are more than kQkvFlags of them,
+// or the RoPE table does not fit in shared memory beside them.
+constexpr int kQkvFlags = 1024;
+cudaError_t launch_qkv_fused(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias,
+                             float* ss, unsigned* flags, unsigned epoch, int tokens, int dim,
+                             int* err, const RopeParams& rp, const QkvOutMaps& om,
+                             cudaStream_t s);
 bool encode_2d_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
                    long long cols, long long rows, int box_cols, int box_rows, char* err,
                    size_t errlen);

@@ -254,10 +254,13 @@ def test_lengths_above_two_to_the_30_are_rejected():
 
 # ------------------------------------------------------------------ q/k/v projection (host checks)
 def test_qkv_workspace_and_host_checks():
-    # y in f32 for 3 * dim features per token, then two sums of squares per token
+    # y in f32 for 3 * dim features per token, two sums of squares per token,
+    # then two arrival counters per block of 256 tokens (the fused launch)
     ws = pv.pv_qkv_ws_bytes(880, 3072)
     y = 880 * 3 * 3072 * 4
-    assert ws == ((y + 255) // 256) * 256 + ((880 * 8 + 255) // 256) * 256
+    r = lambda n: ((n + 255) // 256) * 256
+    # y, then one partial sum of squares per token, q / k and 256-feature tile
+    assert ws == r(y) + r(880 * 2 * 12 * 4)
     for args in ((0, 3072), (880, 100), (880, 0)):
         with pytest.raises(pv.PVError) as e:
             pv.pv_qkv_ws_bytes(*args)

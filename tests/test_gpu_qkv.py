@@ -3,7 +3,9 @@ on the GPU against the fp64 oracle (oracle/projection.py, oracle/rope.py):
 q_rot and the K rows within the bf16 RoPE bound, V rows within half a bf16
 ulp plus the f32 accumulation, rows placed where the schedule puts them, for
 the three GEMM tile widths (dim a multiple of 256, 128 and 64 only) and two
-streams in one call."""
+streams in one call; the one-launch path (every GEMM tile resident, the norm
+and RoPE in the GEMM epilogue) for the small cases and the steady chunk, the
+two-launch path for the profile's first chunk."""
 import numpy as np
 import pytest
 import torch
@@ -110,6 +112,35 @@ def test_steady_chunk_profile(pv):
     st.close()
 
 
+def test_first_chunk_profile_two_launch_path(pv):
+    # the profile's first chunk: 2,640 tokens of dim 3072 need 396 GEMM tiles,
+    # more than can be resident at once, so the call takes the two-launch path
+    # (GEMM writing y and the sums of squares, then the RoPE / append kernel)
+    W, Hh, heads, d, R = 40, 22, 24, 128, 18
+    T = W * Hh
+    n = 3 * T
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B4, 0), (n, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 13)
+    q_rot = torch.empty(heads * n * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(n, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [0], 0, 1, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    rows = np.array([0, 127, 128, 879, 880, 1759, 1760, 2559, 2560, 2639])
+    qr, kr, v = _oracle(x, w, b, g_q, g_k, heads, W, Hh, 0, d, rows)
+    Kr, Vr = st.k_region(), st.v_region()
+    assert_rope_close(f64(q_rot.view(heads, n, d)[:, rows]), qr.transpose(1, 0, 2), "q_rot")
+    assert_rope_close(f64(Kr[0, 1, 0, :, rows]), kr.transpose(1, 0, 2), "K rows")
+    _assert_v_close(f64(Vr[0, 1, 0, :, rows]), v.transpose(1, 0, 2), "V rows")
+    st.close()
+
+
 def test_two_streams_one_call(pv):
     # a stream in its first chunk (96 tokens) and one at a steady chunk (32)
     W, Hh, heads, d, R = 8, 4, 2, 128, 2
@@ -143,6 +174,41 @@ def test_two_streams_one_call(pv):
     r0 = 3 * T + s.slot * T
     assert_rope_close(f64(Kr[0, 1, 1, :, r0:r0 + n1]), kr.transpose(1, 0, 2), "K1")
     _assert_v_close(f64(Vr[0, 1, 1, :, r0:r0 + n1]), v.transpose(1, 0, 2), "V1")
+    st.close()
+
+
+def test_sink_pass_two_streams_boundary_inside_a_warp(pv):
+    # the bootstrap pass of two streams (K/V rows to the sink of all 4 step
+    # buffers) with 60 tokens each: the stream boundary falls inside the
+    # second group of 32 tokens, whose rows are written lane by lane, the
+    # other groups by whole-box stores, each to every step buffer
+    W, Hh, heads, d, R = 5, 4, 2, 128, 2
+    T = W * Hh
+    n = 3 * T
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_streams=2, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    for i in (0, 1):
+        pv.pv_kv_begin_chunk(h, i, 3)
+        pv.pv_kv_begin_sink(h, i)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B5, 0), (2 * n, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 17)
+    q_rot = torch.empty(heads * 2 * n * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(2 * n, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [0, 1], 0, pv.PV_STEP_SINK, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    Kr, Vr = st.k_region(), st.v_region()
+    for i in (0, 1):
+        qr, kr, v = _oracle(x[i * n:(i + 1) * n], w, b, g_q, g_k, heads, W, Hh, 0, d)
+        qi = q_rot[heads * i * n * d:heads * (i + 1) * n * d].view(heads, n, d)
+        assert_rope_close(f64(qi), qr.transpose(1, 0, 2), f"q_rot stream {i}")
+        for s_ in range(4):
+            assert_rope_close(f64(Kr[0, s_, i, :, :n]), kr.transpose(1, 0, 2), f"K stream {i} step {s_}")
+            _assert_v_close(f64(Vr[0, s_, i, :, :n]), v.transpose(1, 0, 2), f"V stream {i} step {s_}")
+            assert int(torch.count_nonzero(Kr[0, s_, i, :, n:])) == 0
     st.close()
 
 
