@@ -82,6 +82,37 @@ def test_first_chunk_tiny(pv, heads, d):
     st.close()
 
 
+@pytest.mark.parametrize("heads,d", [(2, 64), (3, 64), (1, 128)])
+def test_one_launch_several_token_blocks(pv, heads, d):
+    # 3 frames of 13 x 17 = 663 tokens: 3 token blocks of 256 (the last
+    # ragged) x 3 dim / BN feature tiles (dim 128, 192, 128: BN = 128, 64,
+    # 128), all resident at once, so the norm's wait spans several blocks
+    W, Hh, R = 13, 17, 2
+    T = W * Hh
+    n = 3 * T
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B6, heads, d), (n, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 23 + heads * d)
+    q_rot = torch.empty(heads * n * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(n, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    for rep in range(2):  # the second call's flags hold the next epoch
+        q_rot.zero_()
+        pv.pv_qkv_rope_append(h, [0], 0, 3, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+        torch.cuda.synchronize()
+        assert pv.pv_kv_poll_device_error(h) == 0
+        qr, kr, v = _oracle(x, w, b, g_q, g_k, heads, W, Hh, 0, d)
+        Kr, Vr = st.k_region(), st.v_region()
+        assert_rope_close(f64(q_rot.view(heads, n, d)), qr.transpose(1, 0, 2), f"q_rot call {rep}")
+        assert_rope_close(f64(Kr[0, 3, 0, :, :n]), kr.transpose(1, 0, 2), f"K rows call {rep}")
+        _assert_v_close(f64(Vr[0, 3, 0, :, :n]), v.transpose(1, 0, 2), f"V rows call {rep}")
+    st.close()
+
+
 def test_steady_chunk_profile(pv):
     # the profile's steady chunk: 880 tokens of dim 3072 (24 x 128) into ring slot 9
     W, Hh, heads, d, R = 40, 22, 24, 128, 18
