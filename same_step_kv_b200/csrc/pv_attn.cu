@@ -641,6 +641,29 @@ __device__ __forceinline__ void stage_flush(const CUtensorMap* to, const uint8_t
 // are reproducible.  The (m, l) loads are issued four parts at a time (one
 // pass) and a part's 32-column block in one batch: a merge costs a few L2
 // round trips.
+// Split-KV partial rows go to L2 with an evict-last policy, so that the
+// key / value stream of the launch does not push them to DRAM before the
+// last CTA to arrive merges them; that CTA then drops each merged line
+// without writing it back (the next launch writes a slot before it reads
+// it).  Without this about half of the parts written early in a CTA's run
+// went to DRAM and came back; with it the launch's DRAM writes are its
+// output.
+__device__ __forceinline__ unsigned long long l2_keep_policy() {
+    unsigned long long pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void st_keep(float* a, float v, unsigned long long pol) {
+    asm volatile("st.global.cg.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(a), "f"(v), "l"(pol)
+                 : "memory");
+}
+// Drops the 128-byte L2 line at a (128-byte aligned) without writing it
+// back; `after` is computed from the line's data, so that the drop is
+// issued after the line was read.
+__device__ __forceinline__ void l2_discard(const float* a, float after) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(a), "f"(after) : "memory");
+}
+
 template <int D>
 __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, int X, int r,
                                             bool row_ok, bool keep, uint32_t tO, float m_own,
@@ -706,6 +729,15 @@ __device__ __forceinline__ void merge_parts(const AttnParams& p, const Seg& g, i
         }
     }
     if (row_ok && lse_dst) *lse_dst = (M + __log2f(L)) * 0.69314718055994531f;
+    // every part's lines of this warp's 32 rows (the merging CTA's own part
+    // too: it was written before the arrival count and read from TMEM): a
+    // line per lane and 32 columns, then the m and l lines
+    for (int k = 0; k < g.nseg; ++k) {
+        const float* pk = ml(k) - (size_t)kQRows * D;
+        for (int c = 0; c < D; c += 32)
+            l2_discard(pk + (size_t)(c + (r & 31)) * kQRows + (r & ~31), L);
+        if ((r & 31) < 2) l2_discard(ml(k) + (r & 31) * kQRows + (r & ~31), L);
+    }
 }
 
 template <int D, bool kRun>
@@ -819,9 +851,10 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
                     store_row32(dst + c, o, inv);
                 }
             } else {
+                const unsigned long long pol = l2_keep_policy();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    __stcg(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]));
+                    st_keep(mine + (size_t)(c + i) * kQRows + r, __uint_as_float(o[i]), pol);
             }
         }
         if (!keep) {
@@ -834,8 +867,11 @@ __device__ void softmax_epilogue(const AttnParams& p, const CUtensorMap* to, uin
             if (row_ok && p.lse) p.lse[(size_t)tok * p.heads + g.head] = (m + __log2f(l)) * ln2;
             continue;
         }
-        __stcg(mine + (size_t)kQRows * D + r, m);
-        __stcg(mine + (size_t)kQRows * D + kQRows + r, l);
+        {
+            const unsigned long long pol = l2_keep_policy();
+            st_keep(mine + (size_t)kQRows * D + r, m, pol);
+            st_keep(mine + (size_t)kQRows * D + kQRows + r, l, pol);
+        }
         // all four warps' partial rows are visible before the arrival count
         // moves; bounded waits on mbarriers, not bar.sync, so that an
         // aborting CTA can never block here
