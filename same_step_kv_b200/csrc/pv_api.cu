@@ -81,7 +81,7 @@ WsLayout ws_layout(const pv_kv_config& c) {
     w.err_off = 0;
     w.cnt_off = 256;
     w.flag_off = round_up(w.cnt_off + sizeof(int) * (size_t)w.n_counters, 256);
-    w.tab_off = round_up(w.flag_off + sizeof(unsigned) * (size_t)kQkvFlags, 256);
+    w.tab_off = round_up(w.flag_off + sizeof(unsigned long long) * (size_t)kQkvFlags, 256);
     w.part_off = round_up(w.tab_off + sizeof(float2) * (size_t)w.n_table, 256);
     w.total = round_up(w.part_off + sizeof(float) * partial_slot_floats(c.head_dim) *
                                         (size_t)w.n_partials, 256);
@@ -247,8 +247,9 @@ struct pv_kv_s {
     // the K and V regions with 32-row boxes (stores of the fused projection)
     CUtensorMap tm_k32{}, tm_v32{};
     bool maps32 = false;
-    // the last call number of the fused projection (its flags' value)
-    unsigned qkv_epoch = 0;
+    // the last call number of the fused projection (its flags' value; 64
+    // bits, so that it never comes back to a value a stale flag may hold)
+    unsigned long long qkv_epoch = 0;
     std::vector<StreamState> streams;
     std::mutex mu;
     // cached tensor map of the last q_rot buffer
@@ -747,9 +748,8 @@ pv_status pv_qkv_rope_append(pv_kv kv, int n_streams, const int* streams, int la
         om.k = kv->tm_k32;
         om.v = kv->tm_v32;
         // a new value for the flags of this call (0 is the cleared state)
-        unsigned epoch = kv->qkv_epoch + 1;
-        if (epoch == 0) epoch = 1;
-        unsigned* flags = (unsigned*)(kv->ws + kv->wl.flag_off);
+        const unsigned long long epoch = kv->qkv_epoch + 1;
+        unsigned long long* flags = (unsigned long long*)(kv->ws + kv->wl.flag_off);
         e = launch_qkv_fused(tx, tw, bias, ss, flags, epoch, tok, dim, err, p, om, s);
         if (e == cudaSuccess) {
             kv->qkv_epoch = epoch;

@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     qkv_gemm_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                     const __grid_constant__ CUtensorMap ty, const float* __restrict__ bias,
                     float* __restrict__ ss, int tokens, int dim, int* err,
-                    const __grid_constant__ RopeParams rp, unsigned* flags, unsigned epoch,
+                    const __grid_constant__ RopeParams rp, unsigned long long* flags,
+                    unsigned long long epoch,
                     const __grid_constant__ QkvOutMaps om) {
     using C = GCfg<BN>;
     extern __shared__ __align__(1024) uint8_t g_raw[];
@@ -337,15 +338,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
             if (threadIdx.x == 0) {
                 asm volatile("fence.acq_rel.gpu;" ::: "memory");
-                asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flags + cta), "r"(epoch)
+                asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(flags + cta), "l"(epoch)
                              : "memory");
             }
             if (threadIdx.x < nt) {
-                const unsigned* f = flags + (kind * nt + threadIdx.x) * gridDim.x + blockIdx.x;
+                const unsigned long long* f = flags + (kind * nt + threadIdx.x) * gridDim.x + blockIdx.x;
                 const long long w0 = clock64();
                 for (;;) {
-                    unsigned v;
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+                    unsigned long long v;
+                    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
                     if (v == epoch) break;
                     if (*(volatile int*)&b->abort) break;
                     if (clock64() - w0 > kGWait) {
@@ -578,7 +579,7 @@ cudaError_t launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const C
     RopeParams none{};
     QkvOutMaps no_maps{};
     qkv_gemm_kernel<BN, false><<<grid, kGThreads, C::kSmem, s>>>(tx, tw, ty, bias, ss, tokens, dim,
-                                                                 err, none, nullptr, 0u, no_maps);
+                                                                 err, none, nullptr, 0ull, no_maps);
     return cudaGetLastError();
 }
 
@@ -587,9 +588,9 @@ cudaError_t launch_gemm_bn(const CUtensorMap& tx, const CUtensorMap& tw, const C
 // two-launch path).
 template <int BN>
 cudaError_t launch_fused_bn(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias,
-                            float* ss, unsigned* flags, unsigned epoch, int tokens, int dim,
-                            int* err, const RopeParams& rp, const QkvOutMaps& om,
-                            cudaStream_t s) {
+                            float* ss, unsigned long long* flags, unsigned long long epoch,
+                            int tokens, int dim, int* err, const RopeParams& rp,
+                            const QkvOutMaps& om, cudaStream_t s) {
     using C = GCfg<BN>;
     constexpr int kMaxSmem = 227 * 1024;
     static std::atomic<unsigned long long> configured{0};
@@ -636,9 +637,9 @@ cudaError_t launch_qkv_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const 
 }
 
 cudaError_t launch_qkv_fused(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias,
-                             float* ss, unsigned* flags, unsigned epoch, int tokens, int dim,
-                             int* err, const RopeParams& rp, const QkvOutMaps& om,
-                             cudaStream_t s) {
+                             float* ss, unsigned long long* flags, unsigned long long epoch,
+                             int tokens, int dim, int* err, const RopeParams& rp,
+                             const QkvOutMaps& om, cudaStream_t s) {
     switch (qkv_gemm_tile_n(dim)) {
         case 256:
             return launch_fused_bn<256>(tx, tw, bias, ss, flags, epoch, tokens, dim, err, rp, om, s);

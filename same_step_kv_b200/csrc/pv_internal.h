@@ -123,14 +123,14 @@ struct QkvOutMaps {
 // sum of squares per feature tile (no need to clear it); CTA c sets
 // flags[c] = epoch once its partial sums are written, and the CTAs of a
 // token block read them once all of its tiles' flags hold epoch (flags of
-// earlier calls hold other values).  cudaErrorCooperativeLaunchTooLarge when
+// earlier calls hold smaller values: the epoch is a 64-bit call count).  cudaErrorCooperativeLaunchTooLarge when
 // its tiles cannot all be resident, there are more than kQkvFlags of them,
 // or the RoPE table does not fit in shared memory beside them.
 constexpr int kQkvFlags = 1024;
 cudaError_t launch_qkv_fused(const CUtensorMap& tx, const CUtensorMap& tw, const float* bias,
-                             float* ss, unsigned* flags, unsigned epoch, int tokens, int dim,
-                             int* err, const RopeParams& rp, const QkvOutMaps& om,
-                             cudaStream_t s);
+                             float* ss, unsigned long long* flags, unsigned long long epoch,
+                             int tokens, int dim, int* err, const RopeParams& rp,
+                             const QkvOutMaps& om, cudaStream_t s);
 bool encode_2d_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
                    long long cols, long long rows, int box_cols, int box_rows, char* err,
                    size_t errlen);
