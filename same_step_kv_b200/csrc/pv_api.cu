@@ -946,8 +946,8 @@ pv_status pv_attn_dense(const void* q, const void* k, const void* v, int n_q, in
 pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* n_k, int heads,
                                   int head_dim, size_t* ws_bytes) {
     if (!ws_bytes) return fail(PV_ERR_INVALID_ARG, "output pointer is NULL");
-    long long tq, tk;
-    size_t n_cnt, tiles;
+    long long tq = 0, tk = 0;
+    size_t n_cnt = 0, tiles = 0;
     pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, head_dim, &tq, &tk, &n_cnt, &tiles);
     if (st) return st;
     const size_t n_part = 4 * std::min<size_t>(kMaxGrid, std::max<size_t>(tiles, 1));
@@ -959,8 +959,8 @@ pv_status pv_attn_varlen_ws_bytes(int n_seqs, const int* n_q, const int* n_k, in
 pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs, const int* n_q,
                          const int* n_k, int heads, int head_dim, void* out, float* lse, void* ws,
                          size_t ws_bytes, void* cuda_stream) {
-    long long tot_q, tot_k;
-    size_t n_cnt, tiles;
+    long long tot_q = 0, tot_k = 0;
+    size_t n_cnt = 0, tiles = 0;
     pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, head_dim, &tot_q, &tot_k, &n_cnt, &tiles);
     if (st) return st;
     if (tot_q == 0) return PV_OK;  // no queries: nothing to compute
@@ -1021,8 +1021,8 @@ pv_status pv_attn_varlen(const void* q, const void* k, const void* v, int n_seqs
 pv_status pv_attn_plan(int n_seqs, const int* n_q, const int* n_k, int heads, int n_sm,
                        int partial_slots, int* grid, int* mode, long long* ranges) {
     if (!grid || !mode || !ranges) return fail(PV_ERR_INVALID_ARG, "NULL output pointer");
-    long long tot_q, tot_k;
-    size_t n_cnt, tiles;
+    long long tot_q = 0, tot_k = 0;
+    size_t n_cnt = 0, tiles = 0;
     pv_status st = varlen_sizes(n_seqs, n_q, n_k, heads, 128, &tot_q, &tot_k, &n_cnt, &tiles);
     if (st) return st;
     if (tot_q == 0) return fail(PV_ERR_SHAPE, "no queries");
