@@ -82,11 +82,12 @@ def test_first_chunk_tiny(pv, heads, d):
     st.close()
 
 
-@pytest.mark.parametrize("heads,d", [(2, 64), (3, 64), (1, 128)])
+@pytest.mark.parametrize("heads,d", [(2, 64), (3, 64), (1, 128), (4, 64)])
 def test_one_launch_several_token_blocks(pv, heads, d):
     # 3 frames of 13 x 17 = 663 tokens: 3 token blocks of 256 (the last
-    # ragged) x 3 dim / BN feature tiles (dim 128, 192, 128: BN = 128, 64,
-    # 128), all resident at once, so the norm's wait spans several blocks
+    # ragged) x 3 dim / BN feature tiles (dim 128, 192, 128, 256: BN = 128,
+    # 64, 128, 256 with 64-dim heads), all resident at once, so the norm's
+    # wait spans several blocks
     W, Hh, R = 13, 17, 2
     T = W * Hh
     n = 3 * T
@@ -110,6 +111,34 @@ def test_one_launch_several_token_blocks(pv, heads, d):
         assert_rope_close(f64(q_rot.view(heads, n, d)), qr.transpose(1, 0, 2), f"q_rot call {rep}")
         assert_rope_close(f64(Kr[0, 3, 0, :, :n]), kr.transpose(1, 0, 2), f"K rows call {rep}")
         _assert_v_close(f64(Vr[0, 3, 0, :, :n]), v.transpose(1, 0, 2), f"V rows call {rep}")
+    st.close()
+
+
+def test_one_launch_more_than_sixteen_feature_tiles(pv):
+    # 17 heads x 64 = 1,088 features: 64-feature tiles, 17 of them per token
+    # for q and for k, so a token's factor adds 17 partial sums (16 loaded
+    # together, the 17th after); 96 tokens: 51 CTAs, one launch
+    W, Hh, heads, d, R = 8, 4, 17, 64, 2
+    T = W * Hh
+    n = 3 * T
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    pv.pv_kv_begin_chunk(h, 0, 3)
+    dim = heads * d
+    x = synth.normal_bf16(synth.seed_of(0x0B7, 0), (n, dim), "cuda")
+    w, b, g_q, g_k = _weights(heads, d, 29)
+    q_rot = torch.empty(heads * n * d, dtype=torch.bfloat16, device="cuda")
+    wsb = pv.pv_qkv_ws_bytes(n, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    pv.pv_qkv_rope_append(h, [0], 0, 0, x, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    qr, kr, v = _oracle(x, w, b, g_q, g_k, heads, W, Hh, 0, d)
+    Kr, Vr = st.k_region(), st.v_region()
+    assert_rope_close(f64(q_rot.view(heads, n, d)), qr.transpose(1, 0, 2), "q_rot")
+    assert_rope_close(f64(Kr[0, 0, 0, :, :n]), kr.transpose(1, 0, 2), "K rows")
+    _assert_v_close(f64(Vr[0, 0, 0, :, :n]), v.transpose(1, 0, 2), "V rows")
     st.close()
 
 
