@@ -140,14 +140,16 @@ def _hs_worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_head_sharded_two_gloo_ranks_match_one_process():
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_sharded_gloo_ranks_match_one_process(world):
+    # 2 ranks of 2 heads, 4 ranks of 1 head
     import numpy as np
     from oracle.schedule import Geometry
     from oracle.session import SINK_STEP, StreamSession
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_hs_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_hs_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=180) for _ in procs]
@@ -163,7 +165,7 @@ def test_head_sharded_two_gloo_ranks_match_one_process():
         ostep = SINK_STEP if step == "sink" else step
         qq, kk, vv = _hs_inputs(chunk, step, n)
         ref, _ = ses.chunk_attn(0, ostep, ses.rope_append(0, ostep, qq, kk, vv))
-        got = np.concatenate([gathered[r][i] for r in range(2)], axis=0)
+        got = np.concatenate([gathered[r][i] for r in range(world)], axis=0)
         # each head is computed by the same fp64 arithmetic on one rank or the other
         assert np.array_equal(got, ref), (chunk, step)
 
