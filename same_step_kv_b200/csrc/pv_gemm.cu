@@ -334,7 +334,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
             }
             __syncthreads();
             // publish (the fence after the barrier releases every thread's
-            // sums), then thread j < nt waits for tile j of the token block
+            // sums), then thread j < nt waits for tile j of the token block.
+            // A CTA that gave up a wait publishes too: its sums are missing,
+            // but the error word is set and the call's outputs are invalid
+            // either way, and the other CTAs then end without waiting a second
             const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
             if (threadIdx.x == 0) {
                 asm volatile("fence.acq_rel.gpu;" ::: "memory");
