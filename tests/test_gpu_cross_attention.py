@@ -83,6 +83,20 @@ def test_prompt_batch_ragged_text(pv):
     assert torch.equal(got, want)
 
 
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_most_sequences_one_launch(pv, head_dim):
+    # the most sequences one launch takes (PV_MAX_STREAMS = 64), ragged:
+    # queries 0..300 (some sequences skipped), keys 1..700; every row of
+    # both heads against the oracle
+    rng = np.random.default_rng(64 + head_dim)
+    n_q = [int(x) for x in rng.integers(0, 301, size=64)]
+    n_k = [int(x) for x in rng.integers(1, 701, size=64)]
+    n_q[5], n_q[40] = 0, 0
+    n_k[7] = 1
+    qs, ks, vs, out, lse, _ = _run_varlen(pv, n_q, n_k, heads=2, head_dim=head_dim)
+    _check(qs, ks, vs, out, lse, n_q, (0, 1))
+
+
 def test_run_time_hand_out_is_repeatable(pv):
     # short items are handed out at run time from a counter in the workspace
     # (which CTA takes which item depends on timing); the last CTA returns the

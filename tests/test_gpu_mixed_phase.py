@@ -99,3 +99,39 @@ def test_first_and_steady_streams_in_one_call(pv):
             assert_attn_close(f64(out[tok0[i] + rows, hd]), o_ref, f"stream {i} head {hd}")
             assert_lse_close(f64(lse[tok0[i] + rows, hd]), lse_ref, f"stream {i} head {hd}")
     store.close()
+
+
+def test_most_streams_one_call(pv):
+    # the most streams a store holds (PV_MAX_STREAMS = 64), each in its first
+    # chunk (3 frames of 8 x 4 tokens), in one pv_rope_append and one
+    # pv_chunk_attn call; every row of both heads of every eighth stream
+    # against the oracle's rotation and attention
+    from same_step_kv_b200 import synth as sy
+    Wt, Ht, Hs, Ds, S = 8, 4, 2, 64, 64
+    Tt = Wt * Ht
+    n = 3 * Tt
+    cfg = pv.make_config(1, Hs, Ds, Wt, Ht, ring_slots=2, max_streams=S, max_frames=64)
+    store = pv.KVStore(cfg)
+    h = store.handle
+    for i in range(S):
+        pv.pv_kv_begin_chunk(h, i, 3)
+    qkv = [sy.chunk_qkv(i, 0, 1, 0, n, Hs, Ds, "cuda") for i in range(S)]
+    q, k, v = (torch.cat([t[j] for t in qkv]) for j in range(3))
+    q_rot = torch.empty(Hs * S * n * Ds, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(S * n, Hs, Ds, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(S * n, Hs, dtype=torch.float32, device="cuda")
+    streams = list(range(S))
+    pv.pv_rope_append(h, streams, 0, 1, q, k, v, q_rot)
+    pv.pv_chunk_attn(h, streams, 0, 1, q_rot, out, lse)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    f, hh, ww = rope.token_coords(n, Wt, Ht, 0)
+    pairs = rope.axis_pairs(Ds)
+    for i in range(0, S, 8):
+        qr = rope.rotate(f64(qkv[i][0]), f, hh, ww, pairs=pairs)
+        kr = rope.rotate(f64(qkv[i][1]), f, hh, ww, pairs=pairs)
+        for hd in range(Hs):
+            o_ref, lse_ref = attention.attend(qr[:, hd], kr[:, hd], f64(qkv[i][2][:, hd]))
+            assert_attn_close(f64(out[i * n:(i + 1) * n, hd]), o_ref, f"stream {i} head {hd}")
+            assert_lse_close(f64(lse[i * n:(i + 1) * n, hd]), lse_ref, f"stream {i} head {hd}")
+    store.close()
