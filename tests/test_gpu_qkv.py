@@ -201,6 +201,49 @@ def test_first_chunk_profile_two_launch_path(pv):
     st.close()
 
 
+def test_fused_and_two_launch_calls_share_a_handle(pv):
+    # one handle and one workspace: the steady chunk (one launch), then a
+    # 2,640-token first chunk of another stream (two launches, atomics into
+    # the sums after a memset), then the steady chunk again with other
+    # inputs (one launch, the next flag epoch); the last call is checked
+    W, Hh, heads, d, R = 40, 22, 24, 128, 18
+    T = W * Hh
+    cfg = pv.make_config(1, heads, d, W, Hh, ring_slots=R, max_streams=2, max_frames=64)
+    st = pv.KVStore(cfg)
+    h = st.handle
+    s = pv.pv_kv_state()
+    s.phase, s.chunk = pv.PV_PHASE_STEADY, 28
+    pv.pv_kv_set_state(h, 0, s)
+    s = pv.pv_kv_get_state(h, 0)
+    pv.pv_kv_begin_chunk(h, 1, 3)
+    dim = heads * d
+    w, b, g_q, g_k = _weights(heads, d, 31)
+    wsb = pv.pv_qkv_ws_bytes(3 * T, dim)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    q_rot = torch.empty(heads * 3 * T * d, dtype=torch.bfloat16, device="cuda")
+    x0 = synth.normal_bf16(synth.seed_of(0x0B8, 0), (T, dim), "cuda")
+    x1 = synth.normal_bf16(synth.seed_of(0x0B8, 1), (3 * T, dim), "cuda")
+    x2 = synth.normal_bf16(synth.seed_of(0x0B8, 2), (T, dim), "cuda")
+    pv.pv_qkv_rope_append(h, [0], 0, 2, x0, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    pv.pv_qkv_rope_append(h, [1], 0, 2, x1, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    pv.pv_qkv_rope_append(h, [0], 0, 2, x2, w, b, g_q, g_k, EPS, q_rot, ws, wsb)
+    torch.cuda.synchronize()
+    assert pv.pv_kv_poll_device_error(h) == 0
+    rows = np.array([0, 1, 255, 256, 511, 700, 879])
+    qr, kr, v = _oracle(x2, w, b, g_q, g_k, heads, W, Hh, s.frame0, d, rows)
+    r0 = 3 * T + s.slot * T
+    Kr, Vr = st.k_region(), st.v_region()
+    assert_rope_close(f64(q_rot[:heads * T * d].view(heads, T, d)[:, rows]), qr.transpose(1, 0, 2),
+                      "q_rot")
+    assert_rope_close(f64(Kr[0, 2, 0, :, r0 + rows]), kr.transpose(1, 0, 2), "K rows")
+    _assert_v_close(f64(Vr[0, 2, 0, :, r0 + rows]), v.transpose(1, 0, 2), "V rows")
+    # and the first chunk's rows of stream 1 from the two-launch call
+    rows1 = np.array([0, 879, 880, 1759, 2639])
+    qr1, kr1, _ = _oracle(x1, w, b, g_q, g_k, heads, W, Hh, 0, d, rows1)
+    assert_rope_close(f64(Kr[0, 2, 1, :, rows1]), kr1.transpose(1, 0, 2), "stream 1 K rows")
+    st.close()
+
+
 def test_two_streams_one_call(pv):
     # a stream in its first chunk (96 tokens) and one at a steady chunk (32)
     W, Hh, heads, d, R = 8, 4, 2, 128, 2
